@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of one ETA block-sparse decode step on B200.
+
+A step is the whole hot path for one batch of decode queries: threshold
+predictor (Eq. 1) -> block screening against the cached metadata (Eq. 5) ->
+block-sparse flash decoding with the sigmoid logit gate (Eq. 2-3) -> split
+combine. Default workload: GQA decode, batch 8, 32 query / 8 KV heads,
+d=128, 128K cached tokens, bf16 KV, block 32, predictor thresholds at ~38%
+head density (the 128K-context configuration).
+
+Prints one JSON line (rank 0): decode queries/s, effective HBM GB/s on the
+bytes actually read, the decode kernel's roofline fraction, the speedup over
+the same kernel run dense, end-to-end queries/s through the public API with
+host buffers, and the CPU oracle's throughput on a bounded sample.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--density 0.38]
+  python bench.py --impl reference ...   # the CPU oracle as the reference arm
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+L2_FLUSH_BYTES = 512 << 20      # > 2x the 126 MB L2
+LAUNCHES_PER_STEP = {"predictor": 4, "const": 3}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="eta", choices=["eta", "reference"])
+    p.add_argument("--config", type=int, default=3)
+    p.add_argument("--batch", type=int, default=None, help="override the batch (config 5 sweep)")
+    p.add_argument("--density", type=float, default=0.38)
+    p.add_argument("--n-splits", type=int, default=0)
+    p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    p.add_argument("--no-dense", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--sweep", action="store_true", help="also report every density of the configuration")
+    p.add_argument("--cpu-groups", type=int, default=64, help="(b, kv head) groups in the CPU sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ byte models
+def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
+    """Algorithmic bytes of one step from the admitted counts.
+    union_cnt [B][Hkv]; the last block of each list is partial when n % b != 0."""
+    eb = 2 if w.dtype == "bf16" else 4
+    row = w.d * eb
+    last_rows = w.n - (w.nb - 1) * w.bs
+    blocks = int(union_cnt.sum())
+    bh = w.B * w.Hkv
+    kv = 2 * row * (blocks * w.bs - bh * (w.bs - last_rows))
+    lists_read = 4 * blocks
+    q = w.B * w.Hq * w.d * eb
+    T = blocks
+    # partials: one per (query head, range it touches)
+    pre = np.concatenate([[0], np.cumsum(union_cnt.reshape(-1))])
+    slots = 0
+    for i in range(bh):
+        k0 = ((pre[i] + 1) * S - 1) // T
+        k1 = ((pre[i + 1]) * S - 1) // T
+        slots += int(k1 - k0 + 1)
+    partials = slots * w.G * (w.d + 2) * 4
+    decode = kv + lists_read + q * w.Hkv // w.Hkv + partials
+    meta = bh * w.n_screened * (2 * w.d + 1) * 4
+    W = (w.Hq * w.d * w.Hq * 4 + w.Hq * 4) if w.tau_mode == "predictor" else 0
+    step_read = kv + meta + lists_read + q * 2 + W
+    dense_kv = 2 * row * bh * w.n
+    return {"decode_kernel": decode, "step_read": step_read, "kv": kv, "meta": meta,
+            "dense_kv": dense_kv, "union_blocks": blocks,
+            "d_head": float(head_cnt.sum()) / (w.B * w.Hq * w.nb),
+            "d_union": float(blocks) / (bh * w.nb)}
+
+
+# -------------------------------------------------------------- CPU oracle
+def oracle_setup(w, dw_host, groups):
+    """Oracle-side metadata and thresholds for the sampled (b, kv head) groups."""
+    import oracle
+    from learned_block_sparse_b200 import synth
+    q_host, K_host, V_host = dw_host
+    nf = w.n // w.bs
+    pool = cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 1)
+    metas = dict(zip(groups, pool.map(lambda g: oracle.slice_meta(K_host[g[0], g[1]], w.d, w.bs, nf), groups)))
+    qf = oracle.to_f32(q_host)
+    heads = [(b, kvh * w.G + g) for (b, kvh) in groups for g in range(w.G)]
+
+    def sc(bh):
+        b, hq = bh
+        mu, var, mx = metas[(b, hq // w.G)]
+        return oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, float("-inf"))[1]
+    scores = dict(zip(heads, pool.map(sc, heads)))
+    return metas, qf, heads, scores, pool
+
+
+def oracle_thresholds(w, q_host, W, scores, density):
+    import oracle
+    from learned_block_sparse_b200 import synth
+    if w.tau_mode == "const":
+        tau = np.zeros((w.Hq,), np.float32)
+        for h in range(w.Hq):
+            s = [scores[k] for k in scores if k[1] == h]
+            tau[h] = synth.tau_for_density(np.concatenate(s), density) if s else 0.0
+        return ("const", tau, None)
+    tau0 = oracle.predict_tau(q_host, W, np.zeros(w.Hq, np.float32))
+    bias = np.zeros((w.Hq,), np.float32)
+    for h in range(w.Hq):
+        diffs = [synth.tau_for_density(scores[k], density) - tau0[k[0], h] for k in scores if k[1] == h]
+        bias[h] = np.float32(np.median(diffs)) if diffs else 0.0
+    return ("predictor", None, bias)
+
+
+def oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool):
+    """One oracle decode step over the sampled heads: predictor, screen, gated attention."""
+    import oracle
+    kind, tau_c, bias = thr
+    tau = oracle.predict_tau(q_host, W, bias) if kind == "predictor" else None
+
+    def one(bh):
+        b, hq = bh
+        kvh = hq // w.G
+        t = float(tau[b, hq]) if tau is not None else float(tau_c[hq])
+        mu, var, mx = metas[(b, kvh)]
+        lst, _ = oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, t)
+        return oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, w.n, qf[b, hq], lst, t, w.beta)
+    return list(pool.map(one, heads))
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from learned_block_sparse_b200 import synth
+    w = synth.WORKLOADS[args.config]
+    if args.batch:
+        w = w.replace(B=args.batch)
+    rng = np.random.default_rng(0)
+    groups_all = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    n_groups = min(8, len(groups_all))
+    groups = sorted(groups_all[i] for i in rng.choice(len(groups_all), n_groups, replace=False))
+    q_host, K_host, V_host = host_slices(w, groups)
+    W = synth.make_predictor(w)[0].numpy() if w.tau_mode == "predictor" else None
+    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups)
+    thr = oracle_thresholds(w, q_host, W, scores, args.density)
+    for _ in range(args.warmup):
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = len(heads) / dt
+    cores = pool._max_workers
+    line = {"impl": "reference", "metric": "sparse decode queries/s", "value": value, "unit": "queries/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": w.name, "density": args.density, "batch": w.B, "seq_len": w.n},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{len(heads)} decode queries ({n_groups} (batch, kv head) groups) of "
+                                       f"the workload per step"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def host_slices(w, groups):
+    """q for all heads, and K/V host tensors holding (at least) the sampled groups.
+    Only the sampled batches are generated; the others stay empty."""
+    from learned_block_sparse_b200 import synth
+    q = synth.make_q(w)
+    K = torch.empty((w.B, w.Hkv, w.capacity, w.d), dtype=w.torch_dtype)
+    V = torch.empty_like(K)
+    needles = synth.make_needles(w)
+    for b in sorted({g[0] for g in groups}):
+        synth.fill_kv(w, q, "k", K[b:b + 1], b, b + 1, needles)
+        synth.fill_kv(w, q, "v", V[b:b + 1], b, b + 1, needles)
+    return q, K, V
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_eta(args):
+    world, rank, local = dist_setup(args)
+    from learned_block_sparse_b200 import binding, synth
+    from learned_block_sparse_b200.workload import DeviceWorkload
+
+    w = synth.WORKLOADS[args.config]
+    if args.batch:
+        w = w.replace(B=args.batch)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    dw = DeviceWorkload(w, device=dev, n_splits=args.n_splits)
+    dec = dw.dec
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    S = args.n_splits or torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def thresholds(density):
+        tau, stride, bias = dw.calibrate(density)
+        return tau, stride, bias
+
+    def step_phases(tau, stride, bias, ev):
+        """predict (if any) -> screen -> decode+combine, events between phases."""
+        ev[0].record(stream)
+        if bias is not None:
+            binding.predict_tau(dec.shape, dw.q, dw.W, bias, dec.tau)
+            t, s = dec.tau, w.Hq
+        else:
+            t, s = tau, stride
+        ev[1].record(stream)
+        binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, t, s, dec.ws)
+        ev[2].record(stream)
+        binding.decode_screened(dec.shape, dec.params, dw.q, dw.K, dw.V, w.n, t, s, dec.out, dec.ws)
+        ev[3].record(stream)
+
+    def time_sparse(density, sample_clocks=False):
+        tau, stride, bias = thresholds(density)
+        for _ in range(args.warmup):
+            flush.zero_()
+            step_phases(tau, stride, bias, [torch.cuda.Event(enable_timing=True) for _ in range(4)])
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        clk = ClockSampler(local) if sample_clocks else None
+        barrier(world)
+        torch.cuda.synchronize()
+        if clk:
+            clk.start()
+        for i in range(args.steps):
+            flush.zero_()
+            step_phases(tau, stride, bias, evs[i])
+        torch.cuda.synchronize()
+        barrier(world)
+        clocks = clk.stop() if clk else None
+        tot = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
+        pre = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        scr = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+        dec_t = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+        # counts for the byte model (untimed extra screen with count outputs)
+        ucnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=dev)
+        hcnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=dev)
+        if bias is not None:
+            binding.predict_tau(dec.shape, dw.q, dw.W, bias, dec.tau)
+            t, s = dec.tau, w.Hq
+        else:
+            t, s = tau, stride
+        binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, t, s, dec.ws, union_cnt=ucnt,
+                       active_cnt=hcnt)
+        torch.cuda.synchronize()
+        bm = byte_model(w, ucnt.cpu().numpy(), hcnt.cpu().numpy(), S)
+        st = dec.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} after timed steps")
+        return {"ms": tot, "ms_predict": pre, "ms_screen": scr, "ms_decode": dec_t, "bytes": bm,
+                "clocks": clocks, "tau": (tau, stride, bias)}
+
+    def time_dense():
+        for _ in range(args.warmup):
+            flush.zero_()
+            dec.dense(dw.q, dw.K, dw.V, w.n)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            dec.dense(dw.q, dw.K, dw.V, w.n)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+
+    def time_e2e(tau, stride, bias):
+        """Public API (EtaDecoder.step) with q from pinned host memory and the
+        output read back to pinned host memory, every step."""
+        q_pin = dw.q_host.pin_memory()
+        out_pin = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
+        q_dev = torch.empty_like(dw.q)
+        tau_dev = tau
+
+        def one():
+            q_dev.copy_(q_pin, non_blocking=True)
+            if bias is not None:
+                o = dec.step(q_dev, dw.K, dw.V, w.n, W=dw.W, bias=bias)
+            else:
+                o = dec.step(q_dev, dw.K, dw.V, w.n, tau=tau_dev, tau_batch_stride=stride)
+            out_pin.copy_(o, non_blocking=True)
+        for _ in range(args.warmup):
+            flush.zero_()
+            one()
+        torch.cuda.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            one()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        h2d = q_pin.numel() * q_pin.element_size()
+        d2h = out_pin.numel() * out_pin.element_size()
+        return ms, h2d, d2h
+
+    main = time_sparse(args.density, sample_clocks=True)
+    ms = max_over_ranks(main["ms"], world)
+    ms_dec = max_over_ranks(main["ms_decode"], world)
+    queries = w.B * w.Hq
+    value = world * queries / (ms * 1e-3)
+    bm = main["bytes"]
+    peak, peak_kind = measured_peaks()
+    achieved = bm["decode_kernel"] / (ms_dec * 1e-3) / 1e9
+    line = {
+        "metric": "sparse decode queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded Philox4x32-10 + Box-Muller; see DESIGN.md input recipe)",
+        "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
+                   "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
+                   "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
+        "effective_hbm_gbs": bm["step_read"] / (ms * 1e-3) / 1e9,
+        "d_head": bm["d_head"], "d_union": bm["d_union"],
+        "phases_ms": {"predict": main["ms_predict"], "screen": main["ms_screen"],
+                      "decode_combine": main["ms_decode"]},
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel (+combine, timed together)",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind, "traffic": None,
+                     "bytes_per_launch": bm["decode_kernel"]},
+        "gpu_launches": LAUNCHES_PER_STEP[w.tau_mode] * args.steps,
+        "clocks": main["clocks"],
+    }
+    if not args.no_dense:
+        dms = max_over_ranks(time_dense(), world)
+        line["dense"] = {"ms_per_step": dms, "queries_per_s": world * queries / (dms * 1e-3),
+                         "hbm_gbs": bm["dense_kv"] / (dms * 1e-3) / 1e9,
+                         "frac_of_peak": bm["dense_kv"] / (dms * 1e-3) / 1e9 / peak}
+        line["speedup_vs_dense"] = dms / ms
+    if not args.no_e2e:
+        tau, stride, bias = main["tau"]
+        ems, h2d, d2h = time_e2e(tau, stride, bias)
+        ems = max_over_ranks(ems, world)
+        line["e2e"] = {"value": world * queries / (ems * 1e-3), "unit": "queries/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+    if args.sweep:
+        sw = {}
+        for dens in w.densities:
+            r = time_sparse(dens)
+            sw[str(dens)] = {"ms": max_over_ranks(r["ms"], world), "d_head": r["bytes"]["d_head"],
+                             "d_union": r["bytes"]["d_union"],
+                             "effective_hbm_gbs": r["bytes"]["step_read"] / (r["ms"] * 1e-3) / 1e9,
+                             "decode_frac": r["bytes"]["decode_kernel"] / (r["ms_decode"] * 1e-3) / 1e9 / peak}
+        line["sweep"] = sw
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(w, args, dw)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(w, args, dw):
+    """The oracle (as it stands) on a bounded sample of the workload: `cpu_groups`
+    (batch, kv head) groups, all their query heads, one decode step."""
+    from learned_block_sparse_b200 import synth
+    rng = np.random.default_rng(1)
+    groups_all = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    n = min(args.cpu_groups, len(groups_all))
+    groups = sorted(groups_all[i] for i in rng.choice(len(groups_all), n, replace=False))
+    q_host, K_host, V_host = host_slices(w, groups)
+    W = synth.make_predictor(w)[0].numpy() if w.tau_mode == "predictor" else None
+    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups)
+    thr = oracle_thresholds(w, q_host, W, scores, args.density)
+    t0 = time.perf_counter()
+    oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+    dt = time.perf_counter() - t0
+    return {"value": len(heads) / dt, "unit": "queries/s", "cores": pool._max_workers, "kind": "oracle",
+            "sample": f"{len(heads)} decode queries ({n} of {len(groups_all)} (batch, kv head) groups), one step: "
+                      f"predictor + screen + gated attention in C (fp32 decisions, fp64 attention)",
+            "seconds": dt}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_eta(args)
+
+
+if __name__ == "__main__":
+    main()

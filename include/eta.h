@@ -1,0 +1,233 @@
+/*
+ * eta.h — C ABI of libeta.so: B200 (sm_100a) block-sparse decode attention for
+ * Elastic Threshold Attention (ETA).
+ *
+ * Method: "Elastic Threshold Attention: Learned Contextual Sparsity for
+ * Long-Context Decoding" (Haris, Li, Karimzadehgan). Section references below
+ * are to the picx.dev summary of that paper (Methodology §1-§4, Eq. 1-5) and
+ * to the figure captions on the thelatestinai.com page (Figure 1, Figure 6).
+ *
+ * Conventions shared by every entry point
+ *  - Every pointer argument is DEVICE memory owned by the caller, unless the
+ *    argument says "host". The library keeps no allocation of its own; the
+ *    per-call scratch lives in a caller-provided workspace.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns after enqueueing its kernels. Calls
+ *    on distinct streams with distinct workspaces may run concurrently.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    rejected call returns ETA_ERR_INVALID_ARG / ETA_ERR_UNSUPPORTED /
+ *    ETA_ERR_WORKSPACE and enqueues nothing. A failed launch returns
+ *    ETA_ERR_CUDA. Errors detected on the device (a bounded wait that ran
+ *    out) are recorded in the workspace status word: read them with
+ *    eta_read_device_status.
+ *  - Layouts (row-major, innermost last):
+ *      q      [B][Hq][d]          kv_dtype-independent: q_dtype
+ *      K, V   [B][Hkv][capacity][d]  kv_dtype; token s of (b, kv head h) at
+ *                                 ((b*Hkv + h)*capacity + s)*d
+ *      meta   mu, var [B][Hkv][d][nb_cap] fp32 (coordinate-major, so one warp
+ *             lane per block reads coalesced), maxnorm [B][Hkv][nb_cap] fp32,
+ *             nb_cap = capacity / block_size
+ *      tau    thresholds indexed tau[b*tau_batch_stride + h]; a stride of 0
+ *             broadcasts one per-head constant over the batch
+ *      out    [B][Hq][d] fp32
+ *  - n_tokens counts the cached tokens INCLUDING the current one (the cache is
+ *    appended before attention); the current token is t = n_tokens - 1. Query
+ *    head h reads kv head h / (Hq / Hkv) (grouped-query attention).
+ */
+#ifndef ETA_H_
+#define ETA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ETA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define ETA_API __attribute__((visibility("default")))
+#else
+#define ETA_API
+#endif
+
+typedef struct CUstream_st* eta_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  ETA_OK = 0,
+  ETA_ERR_INVALID_ARG = 1,    /* a null pointer, bad size, misaligned pointer */
+  ETA_ERR_UNSUPPORTED = 2,    /* a shape this build has no kernel for */
+  ETA_ERR_WORKSPACE = 3,      /* workspace null, misaligned or too small */
+  ETA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
+  ETA_ERR_DEVICE_TIMEOUT = 5  /* a device-side wait exceeded its limit */
+} eta_status_t;
+
+typedef enum { ETA_F32 = 0, ETA_BF16 = 1 } eta_dtype_t;
+
+/* Problem shape. Supported: head_dim in {64, 128}; block_size in
+ * {16, 32, 64, 128}; n_q_heads a multiple of n_kv_heads with group size
+ * Hq/Hkv in {1, 2, 4, 8}; capacity a positive multiple of block_size;
+ * capacity / block_size < 2^24; dtypes ETA_F32 or ETA_BF16. */
+typedef struct {
+  int32_t batch;        /* B */
+  int32_t n_q_heads;    /* Hq */
+  int32_t n_kv_heads;   /* Hkv */
+  int32_t head_dim;     /* d (d_h) */
+  int32_t block_size;   /* b: tokens per KV block (Methodology §4) */
+  int64_t capacity;     /* tokens allocated per (batch, kv head) */
+  int32_t kv_dtype;     /* eta_dtype_t of K and V */
+  int32_t q_dtype;      /* eta_dtype_t of q */
+} eta_shape_t;
+
+/* Method parameters. */
+typedef struct {
+  float beta;          /* gate temperature of Eq. 2 (the end of its anneal, 5.0) */
+  float z;             /* screening confidence z of Eq. 5 */
+  float offset_a;      /* threshold offset a: the screen compares with tau - a */
+  int32_t n_local;     /* trailing blocks admitted without screening (>= 1; the
+                          last block holds the current token, whose gate Eq. 3
+                          exempts) */
+  int32_t n_splits;    /* decode work ranges (thread blocks); 0 = one per SM */
+} eta_params_t;
+
+/* Block metadata of Methodology §4 ("Dual Probabilistic-Geometric Block
+ * Index"): population centroid, coordinate-wise population variance and
+ * maximum key norm of each full block. Layout in the conventions above. */
+typedef struct {
+  float* mu;
+  float* var;
+  float* maxnorm;
+} eta_meta_t;
+
+/* Optional screening outputs (any field may be NULL).
+ *   active_idx [B][Hq][nb_cap]  ascending admitted block indices per query head
+ *   active_cnt [B][Hq]          their count
+ *   union_list [B][Hkv][nb_cap] ascending blocks admitted by any head of the
+ *                               group, packed (block << 8) | head mask, bit g
+ *                               set when query head h*G + g admitted it
+ *   union_cnt  [B][Hkv]         their count
+ *   scores     [B][Hq][nb_cap]  the Eq. 5 score of every screened block */
+typedef struct {
+  int32_t* active_idx;
+  int32_t* active_cnt;
+  uint32_t* union_list;
+  int32_t* union_cnt;
+  float* scores;
+} eta_screen_out_t;
+
+/* ABI version this library was built with (ETA_ABI_VERSION). */
+ETA_API int eta_abi_version(void);
+
+/* Short static description of a status code. */
+ETA_API const char* eta_status_string(eta_status_t status);
+
+/*
+ * eta_build_block_meta — Methodology §4, block index of Eq. 5: for every
+ * (batch, kv head) and every block j in [blk_begin, blk_end), write
+ *   mu_i  = (sum_r k_ri) / b            (sum in increasing r, fp32)
+ *   var_i = (sum_r (k_ri - mu_i)^2) / b (fused multiply-adds in increasing r)
+ *   M     = sqrt(max_r sum_i k_ri^2)    (fused multiply-adds in increasing i)
+ * over the block's b keys. Call it when blocks become full (after an append);
+ * the partial last block never needs metadata (it is always admitted).
+ *   shape  : the cache shape (q_dtype ignored)
+ *   k      : K cache, kv_dtype, 16-byte aligned
+ *   meta   : outputs; entries of other blocks are left untouched
+ * Errors: ETA_ERR_INVALID_ARG when blk_begin < 0, blk_end > capacity/b or
+ * a pointer is null/misaligned. An empty range is a no-op.
+ */
+ETA_API eta_status_t eta_build_block_meta(const eta_shape_t* shape, const void* k, int64_t blk_begin,
+                                          int64_t blk_end, eta_meta_t meta, eta_stream_t stream);
+
+/*
+ * eta_predict_tau — Methodology §1, Eq. 1: tau[b][h] = qbar_b . W[:, h] + bias[h],
+ * qbar_b the concatenation of the Hq query heads of batch b (length Hq*d).
+ *   q    : [B][Hq][d] q_dtype
+ *   W    : [Hq*d][Hq] fp32 row-major (W[j][h] at j*Hq + h)
+ *   bias : [Hq] fp32
+ *   tau  : [B][Hq] fp32 out
+ * The dot product is summed in a fixed order (32 strided fp32 partials by
+ * fused multiply-add, then a pairwise tree), so equal inputs give equal
+ * thresholds on every run.
+ */
+ETA_API eta_status_t eta_predict_tau(const eta_shape_t* shape, const void* q, const float* W,
+                                     const float* bias, float* tau, eta_stream_t stream);
+
+/* Workspace bytes that eta_screen / eta_decode_sparse / eta_decode_dense need
+ * for this shape (sized for the full capacity) and params (n_splits; 0 is
+ * resolved on the current device). Returns 0 for an invalid shape. */
+ETA_API size_t eta_decode_workspace_bytes(const eta_shape_t* shape, const eta_params_t* params);
+
+/* Clear the workspace's device status word (stream-ordered). Call once after
+ * allocating a workspace; eta_read_device_status clears it as well. */
+ETA_API eta_status_t eta_workspace_init(void* workspace, size_t ws_bytes, eta_stream_t stream);
+
+/*
+ * eta_screen — Methodology §4, Eq. 5 and the admission rule: for each query
+ * head, score every block j < nb - n_local with
+ *   Score = fl(fl(min(A, C)) * s),  A = D + z*sqrt(V),  C = sqrt(Q)*M_j,
+ *   D = sum_i q_i mu_ji, V = sum_i (q_i q_i) var_ji, Q = sum_i q_i q_i
+ * (fused multiply-adds in increasing i, s = 1/sqrt(d) rounded to fp32), and
+ * admit the block unless Score < tau - a. The last n_local blocks are
+ * admitted unscreened. Admitted lists are ascending; the union over a GQA
+ * group is formed for loading (a block is read once if any head of its group
+ * admits it).
+ *   q        : [B][Hq][d]; tau: thresholds (see conventions), fp32
+ *   meta     : written by eta_build_block_meta for every screened block
+ *   out      : optional outputs (may be NULL)
+ *   workspace: at least eta_decode_workspace_bytes, 256-byte aligned
+ */
+ETA_API eta_status_t eta_screen(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                eta_meta_t meta, int64_t n_tokens, const float* tau, int64_t tau_batch_stride,
+                                const eta_screen_out_t* out, void* workspace, size_t ws_bytes,
+                                eta_stream_t stream);
+
+/*
+ * eta_decode_sparse — one decode step of ETA (Figure 1 right, Figure 6):
+ * screen (as eta_screen), then a flash-decoding pass over the admitted blocks
+ * only, then a combine of the split partials. For query head h over the
+ * tokens s < n of its admitted blocks (Eq. 2-3):
+ *   S_s = <q, k_s> / sqrt(d)
+ *   g_s = S_s if s = t, else S_s * sigmoid(beta * (S_s - tau))
+ *   out = sum_s exp(g_s - max g) v_s / sum_s exp(g_s - max g)       (fp32)
+ * The gate uses tau; the screen uses tau - a.
+ *   extra : optional screening outputs (may be NULL)
+ */
+ETA_API eta_status_t eta_decode_sparse(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                       const void* k, const void* v, eta_meta_t meta, int64_t n_tokens,
+                                       const float* tau, int64_t tau_batch_stride, float* out,
+                                       const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
+                                       eta_stream_t stream);
+
+/*
+ * eta_decode_screened — the decode and combine half of eta_decode_sparse:
+ * attend over the union lists that the last eta_screen call wrote into this
+ * workspace. That call must have used the same shape, params, q, n_tokens
+ * and tau (the gate reads tau here); with them, eta_screen followed by
+ * eta_decode_screened gives exactly eta_decode_sparse's result. Lets a caller
+ * inspect the admitted sets (counts, density) before paying for the loads.
+ */
+ETA_API eta_status_t eta_decode_screened(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                         const void* k, const void* v, int64_t n_tokens, const float* tau,
+                                         int64_t tau_batch_stride, float* out, void* workspace, size_t ws_bytes,
+                                         eta_stream_t stream);
+
+/*
+ * eta_decode_dense — the same decode kernel with every block admitted (no
+ * screen, no metadata read). tau may be NULL, meaning -infinity: the gate is
+ * then the identity and the result is plain softmax attention.
+ */
+ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                      const void* k, const void* v, int64_t n_tokens, const float* tau,
+                                      int64_t tau_batch_stride, float* out, void* workspace, size_t ws_bytes,
+                                      eta_stream_t stream);
+
+/* Synchronise `stream`, read the workspace's device status word into *status
+ * (host pointer) and clear it. Returns ETA_ERR_CUDA if the copy fails. */
+ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t stream, eta_status_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ETA_H_ */

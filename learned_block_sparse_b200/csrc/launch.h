@@ -1,0 +1,90 @@
+// Internal interface between the C-ABI layer (api.cpp) and the kernel
+// launchers (*.cu). Not part of the public ABI.
+#pragma once
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "eta.h"
+
+namespace eta {
+
+// Per-call scratch carved out of the caller's workspace.
+struct Workspace {
+  int32_t* status;        // device status word (sticky until read)
+  uint32_t* union_list;   // [B*Hkv][nb_cap] (block << 8) | head mask
+  int32_t* union_cnt;     // [B*Hkv]
+  int32_t* head_cnt;      // [B*Hq]
+  int32_t* prefix;        // [B*Hkv + 1] exclusive prefix of union_cnt (decode -> combine)
+  float* o_part;          // [B*Hq][S][d] unnormalised partial outputs
+  float2* ml_part;        // [B*Hq][S] (running max in log2 units, running sum)
+};
+
+struct WsLayout {
+  size_t status, union_list, union_cnt, head_cnt, prefix, o_part, ml_part, total;
+};
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int d, int64_t nb_cap, int S);
+Workspace ws_carve(void* base, const WsLayout& L);
+
+int device_sm_count();
+int device_max_smem_optin();
+
+// Raise a kernel's dynamic shared memory limit to the device maximum, once per
+// device (`done` is the kernel instance's own flag set).
+inline cudaError_t allow_max_smem(std::atomic<uint64_t>& done, const void* fn) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, device_max_smem_optin());
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+cudaError_t launch_build_meta(const eta_shape_t& s, const void* k, int64_t b0, int64_t b1, const eta_meta_t& m,
+                              cudaStream_t st);
+
+cudaError_t launch_predict(const eta_shape_t& s, const void* q, const float* W, const float* bias, float* tau,
+                           cudaStream_t st);
+
+struct ScreenCall {
+  eta_shape_t shape;
+  float z, offset_a;
+  int n_local;
+  const void* q;
+  eta_meta_t meta;
+  int64_t n;
+  const float* tau;
+  int64_t tau_stride;
+  eta_screen_out_t out;   // optional outputs (fields may be null)
+  Workspace ws;
+};
+cudaError_t launch_screen(const ScreenCall& c, cudaStream_t st);
+
+struct DecodeCall {
+  eta_shape_t shape;
+  float beta;
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t n;
+  const float* tau;        // gate thresholds; null = -inf (dense only)
+  int64_t tau_stride;
+  float* out;
+  Workspace ws;
+  int S;                   // number of work ranges (grid size)
+  bool dense;
+};
+cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st);
+
+// Largest B*Hkv the decode kernel's on-chip prefix table holds.
+constexpr int kMaxBH = 8192;
+// Largest number of 32-block tiles one screening thread block holds.
+constexpr int kMaxScreenTiles = 1024;
+constexpr int kMaxCluster = 8;
+
+}  // namespace eta

@@ -44,8 +44,8 @@ def _load():
                                    ctypes.c_int, ctypes.c_double, ctypes.c_void_p)
     lib.synth_normal_fill.argtypes = [u64, u32, u64, i64, dbl, dbl, i32, vp]
     lib.synth_normal_fill.restype = None
-    lib.synth_fill_kv.argtypes = [u64, u32, u32, i32, i64, i64, i64, i64, i64, i64, dbl,
-                                  vp, i32, i64, vp, i32, dbl, vp]
+    lib.synth_fill_kv.argtypes = [u64, u32, u32, i32, i64, i64, i64, i64, i64, i64, i64, i64,
+                                  dbl, vp, i32, i64, vp, i32, dbl, vp]
     lib.synth_fill_kv.restype = None
     lib.synth_pick_blocks.argtypes = [u64, u32, i64, i32, i64, vp]
     lib.synth_pick_blocks.restype = i32
@@ -172,23 +172,33 @@ def make_needles(w: Workload) -> Optional[torch.Tensor]:
     return out
 
 
+def fill_kv(w: Workload, q: torch.Tensor, which: str, dst: torch.Tensor, b0: int = 0,
+            b1: Optional[int] = None, needles: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Fill ``dst`` ([b1-b0][Hkv][capacity][d], CPU) with batches [b0,b1) of K or V."""
+    lib = _load()
+    b1 = w.B if b1 is None else b1
+    assert dst.shape == (b1 - b0, w.Hkv, w.capacity, w.d) and dst.dtype == w.torch_dtype
+    assert dst.is_contiguous() and not dst.is_cuda
+    is_k = which == "k"
+    if is_k and needles is None:
+        needles = make_needles(w)
+    if w.capacity > w.n:
+        dst[:, :, w.n:, :].zero_()
+    lib.synth_fill_kv(w.seed, STREAM_K if is_k else STREAM_V, STREAM_OFFSET, w.dtype_code, w.B, w.Hkv,
+                      w.n, w.capacity, w.d, w.bs, b0, b1,
+                      w.offset_std if is_k else 0.0,
+                      q.data_ptr(), w.dtype_code, w.Hq,
+                      needles.data_ptr() if (is_k and needles is not None) else None,
+                      w.n_needles if is_k else 0, w.needle_scale, dst.data_ptr())
+    return dst
+
+
 def make_kv(w: Workload, q: torch.Tensor, pin: bool = False):
     """K, V [B][Hkv][capacity][d]; tokens >= n are zero."""
-    lib = _load()
-    needles = make_needles(w)
     out = []
-    for stream in (STREAM_K, STREAM_V):
+    for which in ("k", "v"):
         t = _empty((w.B, w.Hkv, w.capacity, w.d), w.torch_dtype, pin)
-        if w.capacity > w.n:
-            t[:, :, w.n:, :].zero_()
-        is_k = stream == STREAM_K
-        lib.synth_fill_kv(w.seed, stream, STREAM_OFFSET, w.dtype_code, w.B, w.Hkv, w.n,
-                          w.capacity, w.d, w.bs,
-                          w.offset_std if is_k else 0.0,
-                          q.data_ptr(), w.dtype_code, w.Hq,
-                          needles.data_ptr() if (is_k and needles is not None) else None,
-                          w.n_needles if is_k else 0, w.needle_scale, t.data_ptr())
-        out.append(t)
+        out.append(fill_kv(w, q, which, t))
     return out[0], out[1]
 
 

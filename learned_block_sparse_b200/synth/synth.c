@@ -144,7 +144,7 @@ typedef struct {
   uint64_t seed;
   uint32_t stream, off_stream;
   int dtype;
-  int64_t B, H, n, cap, d, bs;
+  int64_t B, H, n, cap, d, bs, b0;
   double offset_std;          /* std of the per-block offset vector (0 = none) */
   const void* q;              /* [B][Hq][d] queries in q_dtype, for needles */
   int q_dtype, Hq;
@@ -160,7 +160,8 @@ static void kv_range(void* p, int64_t lo, int64_t hi) {
   const int G = (int)(c->Hq / c->H);
   double qhat[1024];
   int64_t cur_bh = -1;
-  for (int64_t row = lo; row < hi; ++row) {       /* row = (b*H + h)*n + s */
+  for (int64_t lrow = lo; lrow < hi; ++lrow) {    /* lrow = ((b-b0)*H + h)*n + s */
+    const int64_t row = lrow + c->b0 * c->H * c->n;
     int64_t bh = row / c->n, s = row % c->n;
     int64_t b = bh / c->H, h = bh % c->H;
     int64_t blk = s / c->bs;
@@ -180,7 +181,7 @@ static void kv_range(void* p, int64_t lo, int64_t hi) {
     }
     const uint64_t f0 = (uint64_t)row * (uint64_t)d;
     const uint64_t foff = ((uint64_t)bh * (uint64_t)((c->n + c->bs - 1) / c->bs) + (uint64_t)blk) * (uint64_t)d;
-    const int64_t o = (bh * c->cap + s) * d;
+    const int64_t o = ((bh - c->b0 * c->H) * c->cap + s) * d;
     for (int64_t i = 0; i < d; ++i) {
       double x = normal_at(c->seed, c->stream, f0 + (uint64_t)i);
       if (c->offset_std > 0.0) x += c->offset_std * normal_at(c->seed, c->off_stream, foff + (uint64_t)i);
@@ -191,19 +192,22 @@ static void kv_range(void* p, int64_t lo, int64_t hi) {
 }
 
 /*
- * Fill a KV cache [B][H][cap][d] for tokens [0,n): standard normal entries,
- * plus an optional per-(b,h,block) offset vector ~ N(0, offset_std^2 I)
- * shared by every key of the block, plus needle_scale * q_hat on every key
- * of the listed needle blocks (q_hat = unit vector of the group's first
- * query head). Tokens in [n,cap) are left untouched.
+ * Fill batches [b0,b1) of a KV cache [B][H][cap][d] for tokens [0,n):
+ * standard normal entries, plus an optional per-(b,h,block) offset vector
+ * ~ N(0, offset_std^2 I) shared by every key of the block, plus
+ * needle_scale * q_hat on every key of the listed needle blocks (q_hat = unit
+ * vector of the group's first query head). dst points at batch b0's slice;
+ * tokens in [n,cap) are left untouched. q and needles cover all B batches.
  */
 void synth_fill_kv(uint64_t seed, uint32_t stream, uint32_t off_stream, int dtype,
                    int64_t B, int64_t H, int64_t n, int64_t cap, int64_t d, int64_t bs,
-                   double offset_std, const void* q, int q_dtype, int64_t Hq,
-                   const int32_t* needles, int n_needles, double needle_scale, void* dst) {
-  kv_ctx c = {seed, stream, off_stream, dtype, B, H, n, cap, d, bs, offset_std,
+                   int64_t b0, int64_t b1, double offset_std, const void* q, int q_dtype,
+                   int64_t Hq, const int32_t* needles, int n_needles, double needle_scale,
+                   void* dst) {
+  (void)B;
+  kv_ctx c = {seed, stream, off_stream, dtype, B, H, n, cap, d, bs, b0, offset_std,
               q, q_dtype, (int)Hq, needles, n_needles, needle_scale, dst};
-  parallel_for(B * H * n, kv_range, &c);
+  parallel_for((b1 - b0) * H * n, kv_range, &c);
 }
 
 /*

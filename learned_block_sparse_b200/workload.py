@@ -1,0 +1,102 @@
+"""A synthetic decode workload materialised on the GPU.
+
+Generates q, K, V on the host with the seeded generator (batch slices through
+a pinned staging buffer, so the host never holds the whole cache), uploads
+them, builds the block metadata with ``eta_build_block_meta`` and can
+calibrate thresholds to a target density from the library's own block scores
+(``eta_screen`` with score output), as an offline calibration would.
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import binding, synth
+
+
+class DeviceWorkload:
+    def __init__(self, w: synth.Workload, device="cuda", n_splits: int = 0, offset_a: float = 0.0,
+                 keep_host: bool = False, stage_bytes: int = 1 << 30):
+        self.w = w
+        self.device = torch.device(device)
+        self.q_host = synth.make_q(w)
+        self.q = self.q_host.to(self.device)
+        self.needles = synth.make_needles(w)
+        shp = (w.B, w.Hkv, w.capacity, w.d)
+        self.K = torch.empty(shp, dtype=w.torch_dtype, device=self.device)
+        self.V = torch.empty(shp, dtype=w.torch_dtype, device=self.device)
+        per_b = w.Hkv * w.capacity * w.d * (2 if w.dtype == "bf16" else 4)
+        bchunk = max(1, min(w.B, stage_bytes // max(1, per_b)))
+        self.K_host = self.V_host = None
+        if keep_host:
+            self.K_host, self.V_host = synth.make_kv(w, self.q_host)
+            self.K.copy_(self.K_host)
+            self.V.copy_(self.V_host)
+        else:
+            stage = torch.empty((bchunk,) + shp[1:], dtype=w.torch_dtype).pin_memory()
+            for which, dst in (("k", self.K), ("v", self.V)):
+                for b0 in range(0, w.B, bchunk):
+                    b1 = min(w.B, b0 + bchunk)
+                    buf = stage[:b1 - b0]
+                    synth.fill_kv(w, self.q_host, which, buf, b0, b1, self.needles)
+                    dst[b0:b1].copy_(buf, non_blocking=True)
+                    torch.cuda.current_stream(self.device).synchronize()
+            del stage
+        self.dec = binding.EtaDecoder(w.B, w.Hq, w.Hkv, w.d, w.bs, w.capacity, kv_dtype=w.torch_dtype,
+                                      q_dtype=w.torch_dtype, beta=w.beta, z=w.z, offset_a=offset_a,
+                                      n_local=w.n_local, n_splits=n_splits, device=self.device)
+        self.dec.build_meta(self.K, 0, w.n // w.bs)
+        self.W = self.bias0 = None
+        if w.tau_mode == "predictor":
+            W, b0 = synth.make_predictor(w)
+            self.W, self.bias0 = W.to(self.device), b0.to(self.device)
+
+    # ------------------------------------------------------------ calibration
+    def block_scores(self) -> torch.Tensor:
+        """Eq. 5 scores of every screened block, [B][Hq][n_screened] (fp32)."""
+        w = self.w
+        nb_cap = w.capacity // w.bs
+        scores = torch.full((w.B, w.Hq, nb_cap), float("nan"), dtype=torch.float32, device=self.device)
+        tau = torch.full((w.Hq,), float("-inf"), dtype=torch.float32, device=self.device)
+        binding.screen(self.dec.shape, self.dec.params, self.q, self.dec.meta, w.n, tau, 0, self.dec.ws,
+                       scores=scores)
+        return scores[:, :, :w.n_screened]
+
+    @staticmethod
+    def _kth_largest(s: torch.Tensor, density: float) -> torch.Tensor:
+        m = s.shape[-1]
+        if density >= 1.0 or m == 0:
+            return torch.full(s.shape[:-1], float("-inf"), dtype=torch.float32, device=s.device)
+        k = max(1, int(round(density * m)))
+        return s.topk(k, dim=-1).values[..., -1]
+
+    def calibrate(self, density: float):
+        """Thresholds giving about `density` of the screened blocks per head.
+        Per-head constants: (tau [Hq], stride 0). Predictor: bias shifted so the
+        predicted tau hits the per-(b,h) quantile on the median over the batch;
+        returns (None, None, bias) and the caller runs the predictor."""
+        w = self.w
+        sc = self.block_scores()
+        if w.tau_mode == "const":
+            tau = self._kth_largest(sc.transpose(0, 1).reshape(w.Hq, -1), density).contiguous()
+            return tau, 0, None
+        target = self._kth_largest(sc, density)               # [B][Hq]
+        tau0 = torch.empty((w.B, w.Hq), dtype=torch.float32, device=self.device)
+        binding.predict_tau(self.dec.shape, self.q, self.W, self.bias0, tau0)
+        if density >= 1.0:
+            bias = torch.full((w.Hq,), float("-inf"), dtype=torch.float32, device=self.device)
+        else:
+            bias = (target - tau0).median(dim=0).values.contiguous()
+        return None, None, bias
+
+    # ------------------------------------------------------------- one step
+    def step(self, tau=None, stride=None, bias=None, out=None, **outs) -> torch.Tensor:
+        w = self.w
+        if bias is not None:
+            return self.dec.step(self.q, self.K, self.V, w.n, W=self.W, bias=bias, out=out, **outs)
+        return self.dec.step(self.q, self.K, self.V, w.n, tau=tau, tau_batch_stride=stride, out=out, **outs)
+
+    def dense(self, out=None) -> torch.Tensor:
+        return self.dec.dense(self.q, self.K, self.V, self.w.n, out=out)

@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every entry point include/eta.h declares,
+and rejects bad arguments on the host before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "eta.h")
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"ETA_API\s+[\w\s\*]+?\b(eta_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared()
+    for n in ("eta_build_block_meta", "eta_predict_tau", "eta_decode_sparse", "eta_decode_dense", "eta_screen",
+              "eta_decode_workspace_bytes", "eta_read_device_status", "eta_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from learned_block_sparse_b200 import binding
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (eta_\w+)", out))
+    for n in declared():
+        assert n in exported, n
+        assert hasattr(binding.lib, n)
+    assert set(binding.EXPORTED) == set(declared())
+    # nothing else leaks out of the library's C++ internals as eta_ symbols
+    assert exported == set(declared())
+
+
+def test_abi_version_and_status_strings():
+    from learned_block_sparse_b200 import binding
+    assert binding.lib.eta_abi_version() == 1
+    assert binding.status_string(0) == "ok"
+    assert "workspace" in binding.status_string(3)
+    assert binding.status_string(99) == "unknown status"
+
+
+def _shape(**kw):
+    from learned_block_sparse_b200 import binding
+    d = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, block_size=32, capacity=1024, kv_dtype=1, q_dtype=1)
+    d.update(kw)
+    return binding.Shape(**d)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(head_dim=96), 2), (dict(block_size=48, capacity=960), 2), (dict(n_q_heads=6, n_kv_heads=4), 1),
+    (dict(n_q_heads=32, n_kv_heads=2), 2), (dict(capacity=1000), 1), (dict(batch=0), 1), (dict(kv_dtype=7), 1),
+])
+def test_shape_validation(kw, expect):
+    from learned_block_sparse_b200 import binding
+    s = _shape(**kw)
+    p = binding.make_params()
+    k = ctypes.c_void_p(4096)
+    st = binding.lib.eta_decode_dense(ctypes.byref(s), ctypes.byref(p), k, k, k, 100, None, 0, k, k, 1 << 20, None)
+    assert st == expect
+    assert binding.lib.eta_decode_workspace_bytes(ctypes.byref(s), ctypes.byref(p)) == 0
+
+
+def test_argument_validation_before_launch():
+    from learned_block_sparse_b200 import binding
+    s = _shape()
+    p = binding.make_params()
+    L = binding.lib
+    a16 = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 2)
+    meta = binding.Meta(1 << 20, 1 << 20, 1 << 20)
+    # n_tokens out of range, null and misaligned pointers
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 0, a16, 0, a16, None, a16,
+                               1 << 30, None) == 1
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 2000, a16, 0, a16, None,
+                               a16, 1 << 30, None) == 1
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, bad, a16, meta, 100, a16, 0, a16, None, a16,
+                               1 << 30, None) == 1
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 100, None, 0, a16, None,
+                               a16, 1 << 30, None) == 1
+    # workspace: null, misaligned, too small
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 100, a16, 0, a16, None,
+                               None, 1 << 30, None) == 3
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 100, a16, 0, a16, None,
+                               ctypes.c_void_p((1 << 20) + 16), 1 << 30, None) == 3
+    assert L.eta_decode_sparse(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, 100, a16, 0, a16, None,
+                               a16, 64, None) == 3
+    # params
+    for bad_p in (binding.make_params(beta=0.0), binding.make_params(n_local=0), binding.make_params(n_splits=-1),
+                  binding.make_params(z=float("nan"))):
+        assert L.eta_decode_dense(ctypes.byref(s), ctypes.byref(bad_p), a16, a16, a16, 100, None, 0, a16, a16,
+                                  1 << 30, None) == 1
+    # metadata block range
+    assert L.eta_build_block_meta(ctypes.byref(s), a16, -1, 3, meta, None) == 1
+    assert L.eta_build_block_meta(ctypes.byref(s), a16, 0, 33, meta, None) == 1
+    assert L.eta_build_block_meta(ctypes.byref(s), a16, 5, 5, meta, None) == 0      # empty range: no-op
+    assert L.eta_predict_tau(ctypes.byref(s), None, a16, a16, a16, None) == 1
+    st = ctypes.c_int(0)
+    assert L.eta_read_device_status(None, None, ctypes.byref(st)) == 1
+    assert L.eta_workspace_init(bad, 1 << 20, None) == 3
+
+
+def test_workspace_size_grows_with_splits_and_capacity():
+    from learned_block_sparse_b200 import binding
+    s = _shape()
+    a = binding.workspace_bytes(s, binding.make_params(n_splits=4))
+    b = binding.workspace_bytes(s, binding.make_params(n_splits=8))
+    c = binding.workspace_bytes(_shape(capacity=4096), binding.make_params(n_splits=8))
+    assert a < b < c and a % 256 == 0

@@ -1,0 +1,238 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Lists, counts, scores, metadata and thresholds must match bit for bit;
+outputs within 2e-3 (bf16) / 1e-5 (fp32) max-abs. Reduced sizes span several
+tiles, clusters and split ranges with a ragged tail block; the full-size cases
+run the launch configuration the benchmark times and check every list plus
+sampled outputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from learned_block_sparse_b200 import binding, synth
+from learned_block_sparse_b200.workload import DeviceWorkload
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(w, density=None, n_splits=0, offset_a=0.0, heads=None, dense=False, keep_host=True):
+    dw = DeviceWorkload(w, n_splits=n_splits, offset_a=offset_a, keep_host=keep_host)
+    meta = parity.oracle_meta(w, dw.K_host)
+    density = w.densities[0] if density is None else density
+    tau, stride, bias = parity.oracle_thresholds(w, dw.q_host, meta, density, W=dw.W)
+    all_heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    heads = heads or all_heads
+    gpu = parity.run_gpu(dw, tau, stride, bias=bias)
+    assert gpu["status"] == 0
+    if bias is not None:
+        assert np.array_equal(gpu["tau"].view(np.int32), np.asarray(tau, np.float32).view(np.int32)), \
+            "predicted thresholds differ from the oracle's"
+    orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, stride, heads, offset_a=offset_a)
+    err = parity.compare(w, gpu, orc, heads)
+    res = {"err": err, "gpu": gpu, "dw": dw, "tau": tau, "stride": stride, "meta": meta}
+    if dense:
+        g = parity.run_gpu(dw, None, 0, dense=True)
+        assert g["status"] == 0
+        o = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, None, 0, heads, dense=True)
+        parity.compare(w, g, o, heads, check_lists=False)
+    return res
+
+
+# ------------------------------------------------------------------ metadata
+@pytest.mark.parametrize("dtype,d,bs,n,cap", [
+    ("f32", 64, 16, 1024, None), ("bf16", 128, 32, 32 * 70 + 5, 32 * 80),
+    ("bf16", 64, 64, 64 * 9, None), ("bf16", 128, 128, 128 * 5 + 100, None), ("f32", 128, 64, 64 * 7 + 1, None),
+])
+def test_block_meta_bit_exact(dtype, d, bs, n, cap):
+    w = synth.Workload("m", dtype, 2, 4, 2, d, n, bs, z=1.0, tau_mode="const", densities=(0.5,), seed=31,
+                       offset_std=0.7, cap=cap)
+    dw = DeviceWorkload(w, keep_host=True)
+    nf = w.n // w.bs
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            mu, var, mx = oracle.slice_meta(dw.K_host[b, h], w.d, w.bs, nf)
+            g_mu = dw.dec.mu[b, h, :, :nf].T.contiguous().cpu().numpy()
+            g_var = dw.dec.var[b, h, :, :nf].T.contiguous().cpu().numpy()
+            g_mx = dw.dec.maxnorm[b, h, :nf].cpu().numpy()
+            assert np.array_equal(g_mu.view(np.int32), mu.view(np.int32))
+            assert np.array_equal(g_var.view(np.int32), var.view(np.int32))
+            assert np.array_equal(g_mx.view(np.int32), mx.view(np.int32))
+
+
+def test_block_meta_partial_range_leaves_others():
+    w = synth.Workload("m", "bf16", 1, 2, 2, 128, 64 * 10, 64, z=1.0, tau_mode="const", densities=(0.5,), seed=3)
+    dw = DeviceWorkload(w, keep_host=True)
+    dw.dec.mu.fill_(7.0)
+    dw.dec.build_meta(dw.K, 3, 6)
+    torch.cuda.synchronize()
+    assert torch.all(dw.dec.mu[:, :, :, :3] == 7.0) and torch.all(dw.dec.mu[:, :, :, 6:] == 7.0)
+    mu, _, _ = oracle.slice_meta(dw.K_host[0, 1], w.d, w.bs, 6)
+    assert np.array_equal(dw.dec.mu[0, 1, :, 3:6].T.cpu().numpy(), mu[3:6])
+
+
+# ----------------------------------------------------------------- predictor
+@pytest.mark.parametrize("dtype,B,H,d", [("bf16", 3, 16, 128), ("f32", 2, 12, 64), ("bf16", 1, 32, 128)])
+def test_predict_tau_bit_exact(dtype, B, H, d):
+    g = torch.Generator().manual_seed(B * H + d)
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16 if dtype == "bf16" else torch.float32)
+    W = torch.randn(H * d, H, generator=g) / math.sqrt(d)
+    bias = torch.randn(H, generator=g)
+    shape = binding.make_shape(B, H, H, d, 16, 16, q.dtype, q.dtype)
+    tau = torch.empty(B, H, device="cuda")
+    binding.predict_tau(shape, q.cuda(), W.cuda(), bias.cuda(), tau)
+    ref = oracle.predict_tau(q, W.numpy(), bias.numpy())
+    assert np.array_equal(tau.cpu().numpy().view(np.int32), ref.view(np.int32))
+    tau0 = torch.empty(B, H, device="cuda")
+    binding.predict_tau(shape, q.cuda(), torch.zeros_like(W).cuda(), torch.full((H,), -8.0).cuda(), tau0)
+    assert torch.all(tau0 == -8.0)
+
+
+# ------------------------------------------------------- the five workloads
+def _reduced(i):
+    base = synth.WORKLOADS[i]
+    return {
+        1: base,
+        2: base.replace(Hq=4, Hkv=4, n=64 * 40 + 17),
+        3: base.replace(B=2, Hq=8, Hkv=2, n=32 * 150 + 5),
+        4: base.replace(Hq=4, Hkv=4, n=64 * 100 + 63),
+        5: base.replace(B=3, Hq=4, Hkv=4, n=16 * 300 + 9),
+    }[i]
+
+
+@pytest.mark.parametrize("cfg,density", [(1, 0.40), (2, 0.38), (3, 0.20), (3, 0.38), (3, 0.60), (4, 0.38),
+                                         (5, 0.10), (5, 0.25), (5, 0.38), (5, 0.60), (5, 1.0)])
+def test_workload_parity_reduced(cfg, density):
+    r = _full_check(_reduced(cfg), density, dense=(cfg in (1, 4)))
+    assert r["err"] <= parity.TOL[_reduced(cfg).dtype]
+
+
+@pytest.mark.parametrize("n_splits", [1, 2, 7, 150, 1000])
+def test_split_ranges_any_count(n_splits):
+    w = _reduced(3).replace(B=3)
+    _full_check(w, 0.38, n_splits=n_splits)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_group_sizes(G):
+    w = synth.Workload("g", "bf16", 2, 2 * G, 2, 128, 32 * 40 + 3, 32, z=1.0, tau_mode="const",
+                       densities=(0.3,), seed=40 + G, offset_std=synth.SQRT_HALF)
+    _full_check(w, dense=True)
+
+
+@pytest.mark.parametrize("dtype,d,bs", [("bf16", 64, 16), ("bf16", 64, 128), ("f32", 128, 32), ("f32", 64, 64),
+                                        ("bf16", 128, 128)])
+def test_dtypes_dims_blocks(dtype, d, bs):
+    w = synth.Workload("x", dtype, 2, 4, 2, d, bs * 37 + bs // 2 + 1, bs, z=1.0, tau_mode="const",
+                       densities=(0.35,), seed=7 * d + bs, offset_std=synth.SQRT_HALF)
+    _full_check(w, dense=True)
+
+
+def test_edge_single_token_and_exact_blocks():
+    for n in (1, 16, 17, 32):
+        w = synth.Workload("e", "bf16", 1, 2, 2, 128, n, 16, z=1.0, tau_mode="const", densities=(0.5,), seed=n,
+                           cap=64)
+        _full_check(w, dense=True)
+
+
+def test_edge_n_local_and_offset():
+    w = _reduced(5).replace(n_local=3)
+    _full_check(w, 0.25)
+    w = _reduced(3)
+    _full_check(w, 0.38, offset_a=0.4)
+    _full_check(w, 0.38, offset_a=-0.8)
+
+
+def test_extreme_thresholds():
+    w = _reduced(2)
+    dw = DeviceWorkload(w, keep_host=True)
+    meta = parity.oracle_meta(w, dw.K_host)
+    heads = [(0, h) for h in range(w.Hq)]
+    for t in (float("inf"), float("-inf")):
+        tau = np.full((w.Hq,), t, np.float32)
+        gpu = parity.run_gpu(dw, tau, 0)
+        orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, 0, heads)
+        parity.compare(w, gpu, orc, heads)
+        if t == float("inf"):
+            assert np.all(gpu["active_cnt"] == 1)
+        else:
+            assert np.all(gpu["active_cnt"] == w.nb)
+
+
+def test_dense_equals_softmax_and_sparse_at_minus_inf():
+    w = _reduced(4)
+    dw = DeviceWorkload(w, keep_host=True)
+    dense = dw.dense().clone()
+    tau = torch.full((w.Hq,), float("-inf"), device="cuda")
+    sparse = dw.step(tau=tau, stride=0).clone()
+    torch.cuda.synchronize()
+    assert torch.allclose(dense, sparse, atol=1e-6, rtol=0)
+    for h in range(w.Hq):
+        k = dw.K_host[0, h, :w.n].double()
+        v = dw.V_host[0, h, :w.n].double()
+        qq = dw.q_host[0, h].double()
+        ref = torch.softmax(k @ qq / math.sqrt(w.d), 0) @ v
+        assert torch.max(torch.abs(dense[0, h].cpu().double() - ref)) < 2e-3
+
+
+def test_repeat_calls_identical():
+    w = _reduced(3)
+    dw = DeviceWorkload(w)
+    tau = torch.zeros((w.B, w.Hq), device="cuda")
+    a = dw.step(tau=tau, stride=w.Hq).clone()
+    b = dw.step(tau=tau, stride=w.Hq).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------- full size
+def _sample_heads(w, k, seed=0):
+    rng = np.random.default_rng(seed)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    idx = rng.choice(len(pairs), size=min(k, len(pairs)), replace=False)
+    return sorted(pairs[i] for i in idx)
+
+
+def _full_size(w, density, n_out_heads, list_pairs=None):
+    """Full-size workload: every list/score/count checked on the given (b, kvh)
+    pairs (default all), outputs on sampled heads."""
+    dw = DeviceWorkload(w, keep_host=True)
+    pairs = list_pairs or [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    meta = parity.oracle_meta(w, dw.K_host, pairs)
+    list_heads = [(b, kvh * w.G + g) for (b, kvh) in pairs for g in range(w.G)]
+    tau, stride, bias = parity.oracle_thresholds(w, dw.q_host, meta, density, W=dw.W, heads=list_heads)
+    gpu = parity.run_gpu(dw, tau, stride, bias=bias)
+    assert gpu["status"] == 0
+    if bias is not None:
+        assert np.array_equal(gpu["tau"].view(np.int32), np.asarray(tau, np.float32).view(np.int32))
+    out_heads = set(_sample_heads(w.replace(B=w.B), n_out_heads))
+    out_heads = sorted(h for h in out_heads if (h[0], h[1] // w.G) in set(pairs)) or list_heads[:2]
+    orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, stride, list_heads)
+    # lists for every head, outputs for all of them too (the oracle is threaded)
+    parity.compare(w, gpu, orc, list_heads)
+    dens = gpu["active_cnt"].sum() / (w.B * w.Hq * w.nb)
+    return dens
+
+
+def test_full_size_gqa_128k_bench_config():
+    w = synth.WORKLOADS[3]
+    pairs = [(0, 0), (3, 5), (7, 7)]
+    dens = _full_size(w, 0.38, 0, list_pairs=pairs)
+    assert 0.3 < dens < 0.5
+
+
+def test_full_size_mha_32k_needles():
+    _full_size(synth.WORKLOADS[2], 0.38, 0)
+
+
+def test_full_size_512k_sampled():
+    w = synth.WORKLOADS[4]
+    _full_size(w, 0.38, 0, list_pairs=[(0, 2), (0, 11)])
+
+
+def test_full_size_64k_b16_batch16_sampled():
+    w = synth.WORKLOADS[5].replace(B=16)
+    _full_size(w, 0.25, 0, list_pairs=[(0, 0), (9, 3), (15, 15)])
