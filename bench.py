@@ -170,9 +170,9 @@ def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
     for i in range(bh):
         k0 = ((pre[i] + 1) * S - 1) // T
         k1 = ((pre[i + 1]) * S - 1) // T
-        slots += int(k1 - k0 + 1)
+        slots += sum(1 for k in range(int(k0), int(k1) + 1) if (k * T) // S != ((k + 1) * T) // S)
     partials = slots * w.G * (w.d + 2) * 4
-    decode = kv + lists_read + q * w.Hkv // w.Hkv + partials
+    decode = kv + lists_read + q + partials
     meta = bh * w.n_screened * (2 * w.d + 1) * 4
     W = (w.Hq * w.d * w.Hq * 4 + w.Hq * 4) if w.tau_mode == "predictor" else 0
     step_read = kv + meta + lists_read + q * 2 + W

@@ -1,6 +1,7 @@
 // C-ABI entry points of libeta.so (declared in include/eta.h): host-side
 // validation, workspace carving and dispatch to the kernel launchers.
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -127,6 +128,11 @@ eta_status_t check_decode_shape(const eta_shape_t* s, bool dense) {
                        (dense ? 0 : static_cast<size_t>(BH + 1) * 4) + 64;
   const size_t need = 2 * (2 * tile + 32) + fixed;
   if (need + 1024 > static_cast<size_t>(device_max_smem_optin())) return ETA_ERR_UNSUPPORTED;
+  // bf16 K/V with bf16 q take the tensor-core kernel, whose TMA tensor copies
+  // address cache rows with 32-bit coordinates
+  if (s->kv_dtype == ETA_BF16 && s->q_dtype == ETA_BF16 &&
+      static_cast<int64_t>(BH) * s->capacity > static_cast<int64_t>(INT32_MAX))
+    return ETA_ERR_UNSUPPORTED;
   return ETA_OK;
 }
 

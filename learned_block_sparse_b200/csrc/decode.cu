@@ -10,6 +10,10 @@
 // unnormalised output) per query head; the combine kernel merges a head's
 // partials, which come from consecutive thread blocks.
 //
+// This file holds the CUDA-core consumer (fp32 K/V, or bf16 K/V with fp32
+// queries), the combine kernel and the dispatch; bf16 K/V with bf16 queries
+// go to the tensor-core consumer in decode_mma.cu.
+//
 // Pipeline. Warp 8 is the producer: one lane issues two 1-D TMA bulk copies
 // (K block, V block: b*d contiguous elements each) per admitted block into a
 // ring of shared-memory stages guarded by mbarriers; the copies carry an
@@ -24,10 +28,7 @@
 // Every mbarrier wait is bounded (2 s); on timeout the status word is set,
 // the CTA stops issuing copies, waits for the copies already in flight and
 // finishes with the same control flow, so no thread is left at a barrier.
-#include <cmath>
-
-#include "common.cuh"
-#include "launch.h"
+#include "decode_common.cuh"
 
 namespace eta {
 
@@ -36,37 +37,6 @@ namespace {
 constexpr int kNW = 8;                       // consumer warps
 constexpr int kDecThreads = (kNW + 1) * 32;  // + one producer warp
 constexpr int kCombineWarps = 4;
-
-struct DecodeArgs {
-  const void* k;
-  const void* v;
-  const void* q;
-  const float* tau;
-  const uint32_t* union_list;
-  const int32_t* union_cnt;
-  float* o_part;
-  float2* ml_part;
-  int32_t* prefix_out;
-  int32_t* status;
-  int64_t cap, n, tau_stride;
-  int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
-  float beta, qscale;
-};
-
-__device__ __forceinline__ int find_seg(const int32_t* pre, int BH, int64_t p) {
-  int lo = 0, hi = BH - 1;  // largest i with pre[i] <= p
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pre[mid] <= p) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-// The thread block whose range holds flat position x (ranges [k*T/S, (k+1)*T/S)).
-__device__ __forceinline__ int range_of(int64_t x, int64_t T, int S) {
-  return static_cast<int>(((x + 1) * S - 1) / T);
-}
 
 template <typename KV, int D, int G, bool DENSE>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs a) {
@@ -94,26 +64,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   int* s_abort = reinterpret_cast<int*>(s_ml + kNW * G);
   int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
 
-  if (!DENSE) {
-    // exclusive prefix of the union counts
-    for (int i = tid; i < BH; i += kDecThreads) s_pre[i + 1] = a.union_cnt[i];
-    __syncthreads();
-    if (warp == 0) {
-      int run = 0;
-      for (int base = 0; base < BH; base += 32) {
-        const int i = base + lane;
-        int v = i < BH ? s_pre[i + 1] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int u = __shfl_up_sync(kFull, v, o);
-          if (lane >= o) v += u;
-        }
-        if (i < BH) s_pre[i + 1] = run + v;
-        run += __shfl_sync(kFull, v, 31);
-      }
-      if (lane == 0) s_pre[0] = 0;
-    }
-  }
+  if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kDecThreads);
   if (tid == 0) {
     *s_abort = 0;
     for (int s = 0; s < NST; ++s) {
@@ -144,58 +95,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     const uint64_t pol = l2_policy_evict_first();
     const KV* kb = static_cast<const KV*>(a.k);
     const KV* vb = static_cast<const KV*>(a.v);
-    int it = 0, issued = 0, aborted = 0;
-    for (int64_t base = lo; base < hi && !aborted; base += 32) {
-      const int64_t p = base + lane;
-      int seg = 0;
-      uint32_t e = 0;
-      if (p < hi) {
-        seg = seg_of(p);
-        const int64_t j = p - pre(seg);
-        e = DENSE ? ((static_cast<uint32_t>(j) << 8) | ((1u << G) - 1u))
-                  : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + j);
-      }
-      const int cnt = static_cast<int>(hi - base < 32 ? hi - base : int64_t{32});
-      for (int i = 0; i < cnt; ++i, ++it) {
-        const int seg_i = __shfl_sync(kFull, seg, i);
-        const uint32_t e_i = __shfl_sync(kFull, e, i);
-        if (lane == 0 && !aborted) {
-          const int st = it % NST;
-          const int round = it / NST;
-          if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, a.status)) aborted = 1;
-          if (!aborted) {
-            const int blk = static_cast<int>(e_i >> 8);
-            int rows = 0;
-            if (blk < a.nb) {
-              const int64_t r = a.n - static_cast<int64_t>(blk) * a.bs;
-              rows = r < a.bs ? static_cast<int>(r) : a.bs;
-            } else {
-              atomicExch(a.status, static_cast<int32_t>(ETA_ERR_INVALID_ARG));
-            }
-            s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
-            const uint32_t bytes = static_cast<uint32_t>(rows) * D * EB;
-            if (bytes == 0) {
-              mbar_arrive(&s_full[st]);
-            } else {
-              mbar_arrive_expect_tx(&s_full[st], 2 * bytes);
-              const int64_t off = (static_cast<int64_t>(seg_i) * a.cap + static_cast<int64_t>(blk) * a.bs) * D;
-              bulk_g2s(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes, kb + off, bytes, &s_full[st], pol);
-              bulk_g2s(s_tiles + (static_cast<size_t>(st) * 2 + 1) * tile_bytes, vb + off, bytes, &s_full[st], pol);
-            }
-            issued = it + 1;
-          }
-        }
-        aborted = __shfl_sync(kFull, aborted, 0);
-      }
-    }
-    if (lane == 0 && aborted) {
-      // let the copies already issued land before the CTA can exit
-      for (int j = max(0, issued - NST); j < issued; ++j) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
-      }
-    }
+    auto issue = [&](int st, int seg, int blk, int rows) {
+      const uint32_t bytes = static_cast<uint32_t>(rows) * D * EB;
+      mbar_arrive_expect_tx(&s_full[st], 2 * bytes);
+      const int64_t off = (static_cast<int64_t>(seg) * a.cap + static_cast<int64_t>(blk) * a.bs) * D;
+      bulk_g2s(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes, kb + off, bytes, &s_full[st], pol);
+      bulk_g2s(s_tiles + (static_cast<size_t>(st) * 2 + 1) * tile_bytes, vb + off, bytes, &s_full[st], pol);
+    };
+    producer_loop<G, DENSE>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
     return;
   }
 
@@ -404,8 +311,15 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
   const int k0 = range_of(p0, T, a.S);
   const int nsl = range_of(p1 - 1, T, a.S) - k0 + 1;
   const float2* ml = a.ml_part + static_cast<int64_t>(row) * a.S;
+  // A range k is empty when floor(k*T/S) == floor((k+1)*T/S) (only when T < S):
+  // its thread block wrote no partial, so its slot is skipped.
+  auto empty_range = [&](int s) {
+    const int64_t k = k0 + s;
+    return (k * T) / a.S == ((k + 1) * T) / a.S;
+  };
   float M = -INFINITY;
-  for (int s = lane; s < nsl; s += 32) M = fmaxf(M, ml[s].x);
+  for (int s = lane; s < nsl; s += 32)
+    if (!empty_range(s)) M = fmaxf(M, ml[s].x);
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
   constexpr int PL = D / 32;
@@ -415,6 +329,7 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const Combi
   float L = 0.0f;
   const float* op = a.o_part + static_cast<int64_t>(row) * a.S * D;
   for (int s = 0; s < nsl; ++s) {
+    if (empty_range(s)) continue;
     const float2 v = ml[s];
     const float c = (v.x == -INFINITY) ? 0.0f : exp2f(v.x - M);
     L = fmaf(c, v.y, L);
@@ -447,34 +362,16 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_kernel<KV, D, G, DENSE>));
   if (e != cudaSuccess) return e;
 
-  DecodeArgs a;
-  a.k = c.k;
-  a.v = c.v;
-  a.q = c.q;
-  a.tau = c.tau;
-  a.union_list = c.ws.union_list;
-  a.union_cnt = c.ws.union_cnt;
-  a.o_part = c.ws.o_part;
-  a.ml_part = c.ws.ml_part;
-  a.prefix_out = c.ws.prefix;
-  a.status = c.ws.status;
-  a.cap = s.capacity;
-  a.n = c.n;
-  a.tau_stride = c.tau_stride;
-  a.B = s.batch;
-  a.Hq = s.n_q_heads;
-  a.Hkv = s.n_kv_heads;
-  a.bs = s.block_size;
-  a.nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
-  a.nb_cap = static_cast<int>(s.capacity / s.block_size);
-  a.nstages = nst;
-  a.q_dtype = s.q_dtype;
-  a.beta = c.beta;
-  a.qscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  const DecodeArgs a = make_decode_args(c, nst);
   decode_kernel<KV, D, G, DENSE><<<c.S, kDecThreads, smem, st>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
+  return cudaSuccess;
+}
+
+cudaError_t launch_combine(const DecodeCall& c, cudaStream_t st) {
+  const eta_shape_t& s = c.shape;
   CombineArgs ca;
   ca.o_part = c.ws.o_part;
   ca.ml_part = c.ws.ml_part;
@@ -483,11 +380,13 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   ca.B = s.batch;
   ca.Hq = s.n_q_heads;
   ca.Hkv = s.n_kv_heads;
-  ca.nb = a.nb;
+  ca.nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
   ca.S = c.S;
-  ca.dense = DENSE ? 1 : 0;
+  ca.dense = c.dense ? 1 : 0;
   const int rows = s.batch * s.n_q_heads;
-  combine_kernel<D><<<(rows + kCombineWarps - 1) / kCombineWarps, kCombineWarps * 32, 0, st>>>(ca);
+  const unsigned grid = static_cast<unsigned>((rows + kCombineWarps - 1) / kCombineWarps);
+  if (s.head_dim == 128) combine_kernel<128><<<grid, kCombineWarps * 32, 0, st>>>(ca);
+  else combine_kernel<64><<<grid, kCombineWarps * 32, 0, st>>>(ca);
   return cudaGetLastError();
 }
 
@@ -510,9 +409,15 @@ cudaError_t launch_decode_kd(const DecodeCall& c, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st) {
-  if (c.shape.kv_dtype == ETA_BF16)
-    return c.dense ? launch_decode_kd<Bf16Raw, true>(c, st) : launch_decode_kd<Bf16Raw, false>(c, st);
-  return c.dense ? launch_decode_kd<float, true>(c, st) : launch_decode_kd<float, false>(c, st);
+  cudaError_t e;
+  if (c.shape.kv_dtype == ETA_BF16 && c.shape.q_dtype == ETA_BF16)
+    e = launch_decode_mma(c, st);
+  else if (c.shape.kv_dtype == ETA_BF16)
+    e = c.dense ? launch_decode_kd<Bf16Raw, true>(c, st) : launch_decode_kd<Bf16Raw, false>(c, st);
+  else
+    e = c.dense ? launch_decode_kd<float, true>(c, st) : launch_decode_kd<float, false>(c, st);
+  if (e != cudaSuccess) return e;
+  return launch_combine(c, st);
 }
 
 }  // namespace eta

@@ -1,0 +1,420 @@
+// Tensor-core decode for bf16 K/V and bf16 queries: the same flash-decoding
+// pass as decode.cu (gate of Eq. 2-3, online softmax, flat split of the
+// admitted blocks over thread blocks), with the block-level contractions on
+// mma.sync m16n8k16 bf16 tiles.
+//
+// Why tensor cores here: for a GQA group of G heads each admitted 16 KiB K/V
+// block (b=32, d=128) costs 2*G*b*d multiply-adds; on CUDA cores that is
+// ~1,000+ warp instructions per block at G=4 plus the dot-product reductions,
+// more than the ~3,000 issue slots per SM that one block's share of HBM time
+// (at ~6.5 TB/s) leaves. As m16n8k16 tiles (rows = the G heads of the group,
+// columns = keys or head dims) the same block is 32 QK^T + 64 PV mma
+// instructions and 32 ldmatrix loads, so the kernel stays bound by HBM.
+//
+// Data path. The producer warp issues 2-D TMA tensor copies (boxes of
+// [b rows][64 dims], 128-byte swizzle) of each admitted block's K and V into a
+// ring of stages; with that swizzle the 8 rows an ldmatrix reads sit in 8
+// different bank groups. Consumer warps own whole blocks (position i of the
+// range goes to warp i mod 4): S = Q K^T from ldmatrix'd K fragments, scale,
+// gate, online softmax in log2 units on the accumulator fragments, then
+// O += P V with P split into bf16 high and low parts (two mma each) so the
+// probabilities keep ~16 bits of precision, V from ldmatrix.trans. Rows of the
+// 16-row tiles beyond G are zero and ignored.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "decode_common.cuh"
+
+namespace eta {
+
+namespace {
+
+constexpr int kMW = 4;                       // consumer warps
+constexpr int kMmaThreads = (kMW + 1) * 32;  // + one producer warp
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(tm), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D[16x8] += A[16x16] B[16x8] (bf16 in, fp32 accumulate) where only rows 0-7
+// of A are non-zero: a_lo holds A[row][2q..2q+1], a_hi A[row][8+2q..9+2q]
+// (row = lane/4, q = lane%4); d0, d1 are D[row][2q..2q+1].
+__device__ __forceinline__ void mma_rows8(float& d0, float& d1, uint32_t a_lo, uint32_t a_hi, uint32_t b0,
+                                          uint32_t b1) {
+  [[maybe_unused]] float z2, z3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %10, %11};"
+      : "+f"(d0), "+f"(d1), "=f"(z2), "=f"(z3)
+      : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.0f), "f"(0.0f));
+}
+
+// Byte offset of 16-byte chunk `chunk` (8 dims) of tile row `row` in a tile
+// stored as d/64 boxes of [rows][64] bf16 with the 128-byte TMA swizzle.
+__device__ __forceinline__ uint32_t swz(int rows, int row, int chunk) {
+  return static_cast<uint32_t>((chunk >> 3) * rows * 128 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int D, int G, bool DENSE>
+__global__ void __launch_bounds__(kMmaThreads, 1)
+    decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv) {
+  constexpr int KST = D / 16;  // k-steps of QK^T
+  constexpr int NDT = D / 8;   // n-tiles of PV
+  static_assert(G >= 1 && G <= 8, "group size");
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int BH = a.B * a.Hkv;
+  const int NST = a.nstages;
+  const int bs = a.bs;
+  const uint32_t tile_bytes = static_cast<uint32_t>(bs) * D * 2;
+  unsigned char* s_tiles = smem;
+  uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * tile_bytes);
+  uint64_t* s_empty = s_full + NST;
+  int4* s_info = reinterpret_cast<int4*>(s_empty + NST);
+  float* s_macc = reinterpret_cast<float*>(s_info + NST);  // [kMW][G][D]
+  float* s_mm = s_macc + kMW * G * D;                      // [kMW][G]
+  float* s_ml = s_mm + kMW * G;                            // [kMW][G]
+  int* s_abort = reinterpret_cast<int*>(s_ml + kMW * G);
+  int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
+
+  if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kMmaThreads);
+  if (tid == 0) {
+    *s_abort = 0;
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto pre = [&](int i) -> int64_t {
+    return DENSE ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
+  };
+  auto seg_of = [&](int64_t p) -> int {
+    return DENSE ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
+  };
+  const int64_t T = pre(BH);
+  if (!DENSE && blockIdx.x == 0)
+    for (int i = tid; i <= BH; i += kMmaThreads) a.prefix_out[i] = s_pre[i];
+  const int S = gridDim.x;
+  const int kc = blockIdx.x;
+  const int64_t lo = static_cast<int64_t>(kc) * T / S;
+  const int64_t hi = static_cast<int64_t>(kc + 1) * T / S;
+  if (lo >= hi) return;
+
+  if (warp == kMW) {
+    // ------------------------------------------------------------ producer
+    const uint64_t pol = l2_policy_evict_first();
+    auto issue = [&](int st, int seg, int blk, int /*rows*/) {
+      // whole boxes land even for the partial last block (rows past the
+      // cache end read as zeros, rows past n are masked by the consumer)
+      mbar_arrive_expect_tx(&s_full[st], 2 * tile_bytes);
+      const int y = static_cast<int>(static_cast<int64_t>(seg) * a.cap + static_cast<int64_t>(blk) * bs);
+      unsigned char* kt = s_tiles + static_cast<size_t>(st) * 2 * tile_bytes;
+      unsigned char* vt = kt + tile_bytes;
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h) {
+        tma_load_2d(kt + h * bs * 128, &tmk, h * 64, y, &s_full[st], pol);
+        tma_load_2d(vt + h * bs * 128, &tmv, h * 64, y, &s_full[st], pol);
+      }
+    };
+    producer_loop<G, DENSE>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int row = lane >> 2, qd = lane & 3;
+  const bool live_row = row < G;
+  uint32_t qa[KST][2];
+  float o[NDT][2];
+  float m_r = -INFINITY, l_r = 0.0f, tau_r = 0.0f;
+
+  auto load_q = [&](int seg) {
+    const int b = seg / a.Hkv, kvh = seg % a.Hkv;
+    if (live_row) {
+      const uint16_t* qp =
+          static_cast<const uint16_t*>(a.q) + (static_cast<int64_t>(b) * a.Hq + kvh * G + row) * D;
+#pragma unroll
+      for (int kk = 0; kk < KST; ++kk) {
+        const int c = 16 * kk + 2 * qd;
+        qa[kk][0] = static_cast<uint32_t>(qp[c]) | (static_cast<uint32_t>(qp[c + 1]) << 16);
+        qa[kk][1] = static_cast<uint32_t>(qp[c + 8]) | (static_cast<uint32_t>(qp[c + 9]) << 16);
+      }
+      tau_r = a.tau != nullptr ? a.tau[b * a.tau_stride + kvh * G + row] : -INFINITY;
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < KST; ++kk) qa[kk][0] = qa[kk][1] = 0u;
+      tau_r = 0.0f;
+    }
+    m_r = -INFINITY;
+    l_r = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NDT; ++j) o[j][0] = o[j][1] = 0.0f;
+  };
+
+  auto flush = [&](int seg) {
+    float l = l_r + __shfl_xor_sync(kFull, l_r, 1);
+    l += __shfl_xor_sync(kFull, l, 2);
+    if (live_row) {
+#pragma unroll
+      for (int j = 0; j < NDT; ++j) {
+        s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0];
+        s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1];
+      }
+      if (qd == 0) {
+        s_mm[warp * G + row] = m_r;
+        s_ml[warp * G + row] = l;
+      }
+    }
+    named_barrier_sync(1, kMW * 32);
+    const int b = seg / a.Hkv, kvh = seg % a.Hkv;
+    const int slotk = kc - range_of(pre(seg), T, S);
+    for (int idx = tid; idx < G * D; idx += kMW * 32) {
+      const int g = idx / D, e = idx % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kMW; ++w) M = fmaxf(M, s_mm[w * G + g]);
+      float ov = 0.0f, L = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kMW; ++w) {
+        const float c = M == -INFINITY ? 0.0f : exp2f(s_mm[w * G + g] - M);
+        ov = fmaf(c, s_macc[(w * G + g) * D + e], ov);
+        L = fmaf(c, s_ml[w * G + g], L);
+      }
+      const int64_t prow = (static_cast<int64_t>(b) * a.Hq + kvh * G + g) * S + slotk;
+      a.o_part[prow * D + e] = ov;
+      if (e == 0) a.ml_part[prow] = make_float2(M, L);
+    }
+    named_barrier_sync(1, kMW * 32);
+  };
+
+  auto process = [&](int st, const int4 inf) {
+    const uint32_t kt = smem_u32(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes);
+    const uint32_t vt = kt + tile_bytes;
+    const int rows = inf.z;
+    const bool row_on = live_row && ((static_cast<uint32_t>(inf.y) >> row) & 1u);
+    const int64_t tok0 = static_cast<int64_t>(inf.x) * bs;
+    for (int c0 = 0; c0 < bs; c0 += 32) {
+      const int ntc = (bs - c0) >= 32 ? 4 : (bs - c0) / 8;  // n-tiles of 8 keys in this chunk
+      float s[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s[j][0] = s[j][1] = 0.0f;
+        if (j < ntc) {
+          const int krow = c0 + 8 * j + (lane & 7);
+#pragma unroll
+          for (int k2 = 0; k2 < KST / 2; ++k2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kt + swz(bs, krow, 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
+            mma_rows8(s[j][0], s[j][1], qa[2 * k2][0], qa[2 * k2][1], b0, b1);
+            mma_rows8(s[j][0], s[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], b2, b3);
+          }
+        }
+      }
+      // gate (Eq. 2-3) and online softmax on this thread's row
+      float g[4][2];
+      float bm = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = c0 + 8 * j + 2 * qd + e;
+          float v = -INFINITY;
+          if (j < ntc && row_on && key < rows) {
+            const float Sv = s[j][e] * a.qscale;
+            if (tok0 + key == a.n - 1) {
+              v = Sv * kLog2e;  // the current token is exempt from the gate
+            } else {
+              const float x = a.beta * (Sv - tau_r);
+              v = Sv * __frcp_rn(1.0f + exp2f(-x * kLog2e)) * kLog2e;
+            }
+          }
+          g[j][e] = v;
+          bm = fmaxf(bm, v);
+        }
+      bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 2));
+      const float mn = fmaxf(m_r, bm);
+      float corr = 1.0f, ps = 0.0f;
+      float p[4][2];
+      if (mn != -INFINITY) {
+        corr = exp2f(m_r - mn);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            p[j][e] = exp2f(g[j][e] - mn);
+            ps += p[j][e];
+          }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[j][0] = p[j][1] = 0.0f;
+      }
+      l_r = fmaf(l_r, corr, ps);
+      m_r = mn;
+      if (__any_sync(kFull, corr != 1.0f)) {
+#pragma unroll
+        for (int j = 0; j < NDT; ++j) {
+          o[j][0] *= corr;
+          o[j][1] *= corr;
+        }
+      }
+      // O += P V, P = hi + lo in bf16
+#pragma unroll
+      for (int m2 = 0; m2 < 2; ++m2) {
+        if (2 * m2 < ntc) {
+          const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
+          const uint32_t h1 = pack_bf16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
+          const __nv_bfloat162 hb0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
+          const __nv_bfloat162 hb1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
+          const uint32_t l0 = pack_bf16x2(p[2 * m2][0] - __low2float(hb0), p[2 * m2][1] - __high2float(hb0));
+          const uint32_t l1 =
+              pack_bf16x2(p[2 * m2 + 1][0] - __low2float(hb1), p[2 * m2 + 1][1] - __high2float(hb1));
+          const int vrow = c0 + 16 * m2 + 8 * ((lane >> 3) & 1) + (lane & 7);
+#pragma unroll
+          for (int jd = 0; jd < NDT; jd += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
+            mma_rows8(o[jd][0], o[jd][1], h0, h1, b0, b1);
+            mma_rows8(o[jd][0], o[jd][1], l0, l1, b0, b1);
+            mma_rows8(o[jd + 1][0], o[jd + 1][1], h0, h1, b2, b3);
+            mma_rows8(o[jd + 1][0], o[jd + 1][1], l0, l1, b2, b3);
+          }
+        }
+      }
+    }
+  };
+
+  int cur = seg_of(lo);
+  int64_t eff_end = min(pre(cur + 1), hi);
+  load_q(cur);
+  for (int64_t p = lo + warp;; p += kMW) {
+    // every segment that ends at or before this warp's next position is done
+    // for this warp; all consumer warps flush the same segments in order
+    const int64_t lim = p < hi ? p : hi;
+    bool finished = false;
+    while (eff_end <= lim) {
+      flush(cur);
+      if (eff_end >= hi) {
+        finished = true;
+        break;
+      }
+      do {
+        ++cur;
+      } while (pre(cur + 1) <= eff_end);
+      eff_end = min(pre(cur + 1), hi);
+      load_q(cur);
+    }
+    if (finished || p >= hi) break;
+    const int it = static_cast<int>(p - lo);
+    const int st = it % NST;
+    const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, a.status);
+    if (ok) process(st, s_info[st]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&s_empty[st]);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows][d] bf16 view of a K or V cache, boxes of [bs][64] with 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int bs) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
+  const cuuint32_t estride[2] = {1u, 1u};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G, bool DENSE>
+cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
+  const eta_shape_t& s = c.shape;
+  const int BH = s.batch * s.n_kv_heads;
+  const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
+  const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 +
+                       (DENSE ? 0 : static_cast<size_t>(BH + 1) * sizeof(int32_t)) + 1024;
+  const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
+  const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 512;
+  if (fixed + 2 * per_stage > budget) return cudaErrorInvalidValue;
+  // ~200 KB of stages: the consumer warps hold up to 4, the rest are in flight.
+  const size_t nst_bw = (200 * 1024) / (2 * tile), nst_fit = (budget - fixed) / per_stage;
+  int nst = static_cast<int>(nst_bw < nst_fit ? nst_bw : nst_fit);
+  nst = max(2, min(nst, 24));
+  const size_t smem = static_cast<size_t>(nst) * per_stage + fixed + 64;
+
+  CUtensorMap tmk, tmv;
+  const int64_t rows = static_cast<int64_t>(BH) * s.capacity;
+  if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size))
+    return cudaErrorInvalidValue;
+
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE>));
+  if (e != cudaSuccess) return e;
+  const DecodeArgs a = make_decode_args(c, nst);
+  decode_mma_kernel<D, G, DENSE><<<c.S, kMmaThreads, smem, st>>>(a, tmk, tmv);
+  return cudaGetLastError();
+}
+
+template <int D, bool DENSE>
+cudaError_t launch_mma_g(const DecodeCall& c, cudaStream_t st) {
+  switch (c.shape.n_q_heads / c.shape.n_kv_heads) {
+    case 1: return launch_mma_t<D, 1, DENSE>(c, st);
+    case 2: return launch_mma_t<D, 2, DENSE>(c, st);
+    case 4: return launch_mma_t<D, 4, DENSE>(c, st);
+    case 8: return launch_mma_t<D, 8, DENSE>(c, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_mma(const DecodeCall& c, cudaStream_t st) {
+  if (c.shape.head_dim == 128) return c.dense ? launch_mma_g<128, true>(c, st) : launch_mma_g<128, false>(c, st);
+  return c.dense ? launch_mma_g<64, true>(c, st) : launch_mma_g<64, false>(c, st);
+}
+
+}  // namespace eta

@@ -62,7 +62,11 @@ def oracle_thresholds(w, q_host, meta, density, W=None, heads=None):
     bias = np.zeros((w.Hq,), np.float32)
     for h in range(w.Hq):
         diffs = [synth.tau_for_density(sc[(b, h)], density) - tau0[b, h] for b in range(w.B) if (b, h) in sc]
-        bias[h] = np.float32(np.median(diffs)) if density < 1.0 else -np.inf
+        if density >= 1.0:
+            bias[h] = -np.inf
+        elif diffs:
+            bias[h] = np.float32(np.median(diffs))
+        # heads outside the sampled pairs keep bias 0 (any finite threshold is a valid input)
     tau = oracle.predict_tau(q_host, Wn, bias)
     return tau, w.Hq, bias
 
