@@ -215,8 +215,8 @@ def oracle_thresholds(w, q_host, W, scores, density):
     tau0 = oracle.predict_tau(q_host, W, np.zeros(w.Hq, np.float32))
     bias = np.zeros((w.Hq,), np.float32)
     for h in range(w.Hq):
-        diffs = [synth.tau_for_density(scores[k], density) - tau0[k[0], h] for k in scores if k[1] == h]
-        bias[h] = np.float32(np.median(diffs)) if diffs else 0.0
+        rel = [scores[k].astype(np.float64) - tau0[k[0], h] for k in scores if k[1] == h]
+        bias[h] = synth.tau_for_density(np.concatenate(rel), density) if rel else 0.0
     return ("predictor", None, bias)
 
 

@@ -17,9 +17,11 @@
 // different bank groups. Consumer warps own whole blocks (position i of the
 // range goes to warp i mod 4): S = Q K^T from ldmatrix'd K fragments, scale,
 // gate, online softmax in log2 units on the accumulator fragments, then
-// O += P V with P split into bf16 high and low parts (two mma each) so the
-// probabilities keep ~16 bits of precision, V from ldmatrix.trans. Rows of the
-// 16-row tiles beyond G are zero and ignored.
+// O += P V with P split into bf16 high and low parts so the probabilities keep
+// ~16 bits of precision: the high part sits in tile rows 0-7 and the low part
+// in rows 8-15 of the same A operand (G <= 8), so one mma per (k-step, n-tile)
+// accumulates both and the two halves are summed when a partial is emitted.
+// V comes from ldmatrix.trans. In QK^T, rows of the tiles beyond G are zero.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -73,6 +75,28 @@ __device__ __forceinline__ void mma_rows8(float& d0, float& d1, uint32_t a_lo, u
 // stored as d/64 boxes of [rows][64] bf16 with the 128-byte TMA swizzle.
 __device__ __forceinline__ uint32_t swz(int rows, int row, int chunk) {
   return static_cast<uint32_t>((chunk >> 3) * rows * 128 + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+// D[16x8] += A[16x16] B[16x8] with all four A registers and accumulators.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -155,7 +179,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
   const int row = lane >> 2, qd = lane & 3;
   const bool live_row = row < G;
   uint32_t qa[KST][2];
-  float o[NDT][2];
+  float o[NDT][4];  // [n-tile][c0 c1 = high part of row, c2 c3 = low part]
   float m_r = -INFINITY, l_r = 0.0f, tau_r = 0.0f;
 
   auto load_q = [&](int seg) {
@@ -178,7 +202,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     m_r = -INFINITY;
     l_r = 0.0f;
 #pragma unroll
-    for (int j = 0; j < NDT; ++j) o[j][0] = o[j][1] = 0.0f;
+    for (int j = 0; j < NDT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
   };
 
   auto flush = [&](int seg) {
@@ -187,8 +211,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     if (live_row) {
 #pragma unroll
       for (int j = 0; j < NDT; ++j) {
-        s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0];
-        s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1];
+        s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0] + o[j][2];
+        s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1] + o[j][3];
       }
       if (qd == 0) {
         s_mm[warp * G + row] = m_r;
@@ -255,7 +279,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
               v = Sv * kLog2e;  // the current token is exempt from the gate
             } else {
               const float x = a.beta * (Sv - tau_r);
-              v = Sv * __frcp_rn(1.0f + exp2f(-x * kLog2e)) * kLog2e;
+              v = Sv * rcp_approx(1.0f + ex2_approx(-x * kLog2e)) * kLog2e;
             }
           }
           g[j][e] = v;
@@ -267,12 +291,12 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       float corr = 1.0f, ps = 0.0f;
       float p[4][2];
       if (mn != -INFINITY) {
-        corr = exp2f(m_r - mn);
+        corr = ex2_approx(m_r - mn);
 #pragma unroll
         for (int j = 0; j < 4; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            p[j][e] = exp2f(g[j][e] - mn);
+            p[j][e] = ex2_approx(g[j][e] - mn);
             ps += p[j][e];
           }
       } else {
@@ -286,6 +310,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         for (int j = 0; j < NDT; ++j) {
           o[j][0] *= corr;
           o[j][1] *= corr;
+          o[j][2] *= corr;
+          o[j][3] *= corr;
         }
       }
       // O += P V, P = hi + lo in bf16
@@ -304,10 +330,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           for (int jd = 0; jd < NDT; jd += 2) {
             uint32_t b0, b1, b2, b3;
             ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
-            mma_rows8(o[jd][0], o[jd][1], h0, h1, b0, b1);
-            mma_rows8(o[jd][0], o[jd][1], l0, l1, b0, b1);
-            mma_rows8(o[jd + 1][0], o[jd + 1][1], h0, h1, b2, b3);
-            mma_rows8(o[jd + 1][0], o[jd + 1][1], l0, l1, b2, b3);
+            // A rows 0-7: high part, rows 8-15: low part of the same P row
+            mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
+            mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
           }
         }
       }

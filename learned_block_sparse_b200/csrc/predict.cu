@@ -1,7 +1,10 @@
 // Threshold predictor (Methodology §1, Eq. 1): tau_h = qbar . W[:, h] + b_h,
-// qbar the concatenation of all query heads. One warp per (batch, head); lane l
-// folds the terms j = l (mod 32) in increasing j, then a butterfly sums the
-// 32 partials, so the result does not depend on the launch.
+// qbar the concatenation of all query heads. The dot product has one fixed
+// order: 32 running partials, partial l folding the terms j = l (mod 32) in
+// increasing j by fused multiply-add, then a butterfly over the 32 partials.
+// A thread block covers one batch row and up to 32 heads: thread (warp l,
+// lane h) folds partial l of head h, so every load of W reads 32 consecutive
+// heads of one row (coalesced); then warp h adds up head h's partials.
 #include "common.cuh"
 #include "launch.h"
 
@@ -9,28 +12,33 @@ namespace eta {
 
 namespace {
 
-constexpr int kPredWarps = 8;
-
-__global__ void __launch_bounds__(kPredWarps * 32)
+__global__ void __launch_bounds__(1024)
     predict_kernel(const void* __restrict__ q, int q_dtype, const float* __restrict__ W,
                    const float* __restrict__ bias, float* __restrict__ tau, int Hq, int D) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y * kPredWarps + warp;
-  if (h >= Hq) return;
+  __shared__ float part[32][33];
+  const int l = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * 32 + lane;
   const int64_t b = blockIdx.x;
   const int64_t Hd = static_cast<int64_t>(Hq) * D;
   float p = 0.0f;
-  for (int64_t j = lane; j < Hd; j += 32) p = __fmaf_rn(load_elem(q, q_dtype, b * Hd + j), __ldg(W + j * Hq + h), p);
-  for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(kFull, p, o));
-  if (lane == 0) tau[b * Hq + h] = __fadd_rn(p, __ldg(bias + h));
+  if (h < Hq) {
+    for (int64_t j = l; j < Hd; j += 32) p = __fmaf_rn(load_elem(q, q_dtype, b * Hd + j), __ldg(W + j * Hq + h), p);
+  }
+  part[l][lane] = p;
+  __syncthreads();
+  const int hh = blockIdx.y * 32 + l;   // warp l now sums head hh
+  float v = part[lane][l];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, o));
+  if (lane == 0 && hh < Hq) tau[b * Hq + hh] = __fadd_rn(v, __ldg(bias + hh));
 }
 
 }  // namespace
 
 cudaError_t launch_predict(const eta_shape_t& s, const void* q, const float* W, const float* bias, float* tau,
                            cudaStream_t st) {
-  dim3 grid(static_cast<unsigned>(s.batch), static_cast<unsigned>((s.n_q_heads + kPredWarps - 1) / kPredWarps));
-  predict_kernel<<<grid, kPredWarps * 32, 0, st>>>(q, s.q_dtype, W, bias, tau, s.n_q_heads, s.head_dim);
+  dim3 grid(static_cast<unsigned>(s.batch), static_cast<unsigned>((s.n_q_heads + 31) / 32));
+  predict_kernel<<<grid, 1024, 0, st>>>(q, s.q_dtype, W, bias, tau, s.n_q_heads, s.head_dim);
   return cudaGetLastError();
 }
 

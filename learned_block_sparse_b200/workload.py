@@ -73,22 +73,21 @@ class DeviceWorkload:
         return s.topk(k, dim=-1).values[..., -1]
 
     def calibrate(self, density: float):
-        """Thresholds giving about `density` of the screened blocks per head.
-        Per-head constants: (tau [Hq], stride 0). Predictor: bias shifted so the
-        predicted tau hits the per-(b,h) quantile on the median over the batch;
-        returns (None, None, bias) and the caller runs the predictor."""
+        """Thresholds admitting about `density` of each head's screened blocks,
+        pooled over the batch. Per-head constants: (tau [Hq], stride 0).
+        Predictor: returns (None, None, bias) with the bias shifted so that
+        score >= q.W + bias holds for that fraction; the caller runs the predictor."""
         w = self.w
         sc = self.block_scores()
         if w.tau_mode == "const":
             tau = self._kth_largest(sc.transpose(0, 1).reshape(w.Hq, -1), density).contiguous()
             return tau, 0, None
-        target = self._kth_largest(sc, density)               # [B][Hq]
         tau0 = torch.empty((w.B, w.Hq), dtype=torch.float32, device=self.device)
         binding.predict_tau(self.dec.shape, self.q, self.W, self.bias0, tau0)
-        if density >= 1.0:
-            bias = torch.full((w.Hq,), float("-inf"), dtype=torch.float32, device=self.device)
-        else:
-            bias = (target - tau0).median(dim=0).values.contiguous()
+        # bias_h: the threshold, relative to each row's predicted tau, that admits
+        # the target fraction of the head's screened blocks pooled over the batch
+        shifted = (sc - tau0[:, :, None]).transpose(0, 1).reshape(w.Hq, -1)
+        bias = self._kth_largest(shifted, density).contiguous()
         return None, None, bias
 
     # ------------------------------------------------------------- one step

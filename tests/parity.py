@@ -61,11 +61,10 @@ def oracle_thresholds(w, q_host, meta, density, W=None, heads=None):
     tau0 = oracle.predict_tau(q_host, Wn, np.zeros(w.Hq, np.float32))
     bias = np.zeros((w.Hq,), np.float32)
     for h in range(w.Hq):
-        diffs = [synth.tau_for_density(sc[(b, h)], density) - tau0[b, h] for b in range(w.B) if (b, h) in sc]
-        if density >= 1.0:
-            bias[h] = -np.inf
-        elif diffs:
-            bias[h] = np.float32(np.median(diffs))
+        # pooled over the batch: scores relative to each row's predicted tau
+        rel = [sc[(b, h)].astype(np.float64) - tau0[b, h] for b in range(w.B) if (b, h) in sc]
+        if rel:
+            bias[h] = synth.tau_for_density(np.concatenate(rel), density)
         # heads outside the sampled pairs keep bias 0 (any finite threshold is a valid input)
     tau = oracle.predict_tau(q_host, Wn, bias)
     return tau, w.Hq, bias

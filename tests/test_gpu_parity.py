@@ -213,7 +213,7 @@ def _full_size(w, density, n_out_heads, list_pairs=None):
     orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, stride, list_heads)
     # lists for every head, outputs for all of them too (the oracle is threaded)
     parity.compare(w, gpu, orc, list_heads)
-    dens = gpu["active_cnt"].sum() / (w.B * w.Hq * w.nb)
+    dens = sum(int(gpu["active_cnt"][b, h]) for (b, h) in list_heads) / (len(list_heads) * w.nb)
     return dens
 
 
