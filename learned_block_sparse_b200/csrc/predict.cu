@@ -22,7 +22,20 @@ __global__ void __launch_bounds__(1024)
   const int64_t Hd = static_cast<int64_t>(Hq) * D;
   float p = 0.0f;
   if (h < Hq) {
-    for (int64_t j = l; j < Hd; j += 32) p = __fmaf_rn(load_elem(q, q_dtype, b * Hd + j), __ldg(W + j * Hq + h), p);
+    // loads of a chunk are issued together; the multiply-adds stay in increasing j
+    constexpr int kChunk = 16;
+    for (int64_t j0 = l; j0 < Hd; j0 += 32 * kChunk) {
+      float qv[kChunk], wv[kChunk];
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c) {
+        const int64_t j = j0 + 32 * c;
+        qv[c] = j < Hd ? load_elem(q, q_dtype, b * Hd + j) : 0.0f;
+        wv[c] = j < Hd ? __ldg(W + j * Hq + h) : 0.0f;
+      }
+#pragma unroll
+      for (int c = 0; c < kChunk; ++c)
+        if (j0 + 32 * c < Hd) p = __fmaf_rn(qv[c], wv[c], p);
+    }
   }
   part[l][lane] = p;
   __syncthreads();

@@ -54,8 +54,9 @@ def oracle_thresholds(w, q_host, meta, density, W=None, heads=None):
     if w.tau_mode == "const":
         tau = np.zeros((w.Hq,), np.float32)
         for h in range(w.Hq):
-            s = np.concatenate([sc[(b, h)] for b in range(w.B) if (b, h) in sc])
-            tau[h] = synth.tau_for_density(s, density)
+            s = [sc[(b, h)] for b in range(w.B) if (b, h) in sc]
+            # heads outside the sampled pairs keep 0 (any finite threshold is a valid input)
+            tau[h] = synth.tau_for_density(np.concatenate(s), density) if s else 0.0
         return tau, 0, None
     Wn = W.cpu().numpy()
     tau0 = oracle.predict_tau(q_host, Wn, np.zeros(w.Hq, np.float32))
