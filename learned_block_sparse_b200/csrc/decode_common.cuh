@@ -64,33 +64,45 @@ __device__ __forceinline__ void block_prefix(const int32_t* cnt, int32_t* s_pre,
   }
 }
 
-// Producer warp: walk positions [lo, hi) in order; for each, wait until its
-// stage is free, publish (block, head mask, rows, segment) in s_info and call
+// Producer warp: walk positions [lo, hi) in order. Lanes 0..PL-1 each take
+// every PL-th position (position lo + i goes to lane i % PL, PL = 4, or less
+// when the ring has fewer stages, so PL consecutive positions never share a
+// stage and are armed in parallel): wait until the position's stage is free,
+// publish (block, head mask, rows, segment) in s_info and call
 // issue(stage, segment, block, rows), which must arm s_full[stage] (arrive +
-// expected bytes) and start the copies. Lane 0 issues; the warp reads the
-// union list 32 entries at a time. A stage's r-th reuse waits for the
+// expected bytes) and start the copies. The warp reads the union list 32
+// entries at a time, one batch ahead. A stage's r-th reuse waits for the
 // consumer release that completed the empty barrier's phase r-1.
 template <int G, bool DENSE, typename SegOf, typename Pre, typename Issue>
 __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, int64_t hi, int NST,
                                               uint64_t* s_empty, int4* s_info, int* s_abort, SegOf seg_of,
                                               Pre pre, Issue issue, uint64_t* s_full) {
+  const int PL = NST >= 4 ? 4 : (NST >= 2 ? 2 : 1);  // issuing lanes
   const int lane = threadIdx.x & 31;
-  int it = 0, issued = 0, aborted = 0;
-  for (int64_t base = lo; base < hi && !aborted; base += 32) {
-    const int64_t p = base + lane;
-    int seg = 0;
-    uint32_t e = 0;
+  auto load_entry = [&](int64_t p, int& seg, uint32_t& e) {
+    seg = 0;
+    e = 0;
     if (p < hi) {
       seg = seg_of(p);
       const int64_t j = p - pre(seg);
       e = DENSE ? ((static_cast<uint32_t>(j) << 8) | ((1u << G) - 1u))
                 : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + j);
     }
+  };
+  int seg_cur, seg_nxt = 0;
+  uint32_t e_cur, e_nxt = 0;
+  load_entry(lo + lane, seg_cur, e_cur);
+  int issued = 0;    // this lane: 1 + the last position (relative to lo) it armed
+  int aborted = 0;
+  for (int64_t base = lo; base < hi && !aborted; base += 32) {
+    if (base + 32 < hi) load_entry(base + 32 + lane, seg_nxt, e_nxt);
     const int cnt = static_cast<int>(hi - base < 32 ? hi - base : int64_t{32});
-    for (int i = 0; i < cnt; ++i, ++it) {
-      const int seg_i = __shfl_sync(kFull, seg, i);
-      const uint32_t e_i = __shfl_sync(kFull, e, i);
-      if (lane == 0 && !aborted) {
+    for (int s = 0; s < cnt && !aborted; s += PL) {
+      const int src = s + (lane < PL ? lane : 0);
+      const int seg_i = __shfl_sync(kFull, seg_cur, src);
+      const uint32_t e_i = __shfl_sync(kFull, e_cur, src);
+      if (lane < PL && src < cnt) {
+        const int it = static_cast<int>(base - lo) + src;
         const int st = it % NST;
         const int round = it / NST;
         if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, a.status)) aborted = 1;
@@ -109,12 +121,14 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
           issued = it + 1;
         }
       }
-      aborted = __shfl_sync(kFull, aborted, 0);
+      aborted = __any_sync(kFull, aborted) ? 1 : 0;
     }
+    seg_cur = seg_nxt;
+    e_cur = e_nxt;
   }
-  if (lane == 0 && aborted) {
-    // let the copies already issued land before the thread block can exit
-    for (int j = max(0, issued - NST); j < issued; ++j) {
+  if (aborted && lane < PL) {
+    // let the copies this lane armed land before the thread block can exit
+    for (int j = issued - 1; j >= 0 && j >= issued - NST; j -= PL) {
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
       }

@@ -104,13 +104,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int D, int G, bool DENSE>
+template <int D, int G, bool DENSE, int CH>
 __global__ void __launch_bounds__(kMmaThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   constexpr int KST = D / 16;  // k-steps of QK^T
   constexpr int NDT = D / 8;   // n-tiles of PV
   static_assert(G >= 1 && G <= 8, "group size");
+  static_assert(CH == 16 || CH == 32, "keys per chunk");
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -241,59 +242,74 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     named_barrier_sync(1, kMW * 32);
   };
 
+  // gate in log2 units: g = S * sigmoid(beta (S - tau)) * log2(e)
+  const float nbl = -a.beta * kLog2e;
+  auto gate = [&](float Sv) { return Sv * rcp_approx(1.0f + ex2_approx(nbl * (Sv - tau_r))) * kLog2e; };
+
   auto process = [&](int st, const int4 inf) {
     const uint32_t kt = smem_u32(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes);
     const uint32_t vt = kt + tile_bytes;
     const int rows = inf.z;
     const bool row_on = live_row && ((static_cast<uint32_t>(inf.y) >> row) & 1u);
     const int64_t tok0 = static_cast<int64_t>(inf.x) * bs;
-    for (int c0 = 0; c0 < bs; c0 += 32) {
-      const int ntc = (bs - c0) >= 32 ? 4 : (bs - c0) / 8;  // n-tiles of 8 keys in this chunk
-      float s[4][2];
+    // full block that does not hold the current token: no per-key checks
+    const bool fast = rows == bs && tok0 + bs <= a.n - 1;
+    constexpr int NT = CH / 8;  // n-tiles of 8 keys per chunk
+    for (int c0 = 0; c0 < bs; c0 += CH) {
+      // S = Q K^T: even and odd k-steps accumulate separately (shorter mma chains)
+      float se[NT][2], so[NT][2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        s[j][0] = s[j][1] = 0.0f;
-        if (j < ntc) {
-          const int krow = c0 + 8 * j + (lane & 7);
+      for (int j = 0; j < NT; ++j) se[j][0] = se[j][1] = so[j][0] = so[j][1] = 0.0f;
 #pragma unroll
-          for (int k2 = 0; k2 < KST / 2; ++k2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kt + swz(bs, krow, 4 * k2 + (lane >> 3)), b0, b1, b2, b3);
-            mma_rows8(s[j][0], s[j][1], qa[2 * k2][0], qa[2 * k2][1], b0, b1);
-            mma_rows8(s[j][0], s[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], b2, b3);
-          }
-        }
+      for (int k2 = 0; k2 < KST / 2; ++k2) {
+        uint32_t bb[NT][4];
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k2 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+                  bb[j][3]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) mma_rows8(se[j][0], se[j][1], qa[2 * k2][0], qa[2 * k2][1], bb[j][0], bb[j][1]);
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+          mma_rows8(so[j][0], so[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], bb[j][2], bb[j][3]);
       }
       // gate (Eq. 2-3) and online softmax on this thread's row
-      float g[4][2];
+      float g[NT][2];
       float bm = -INFINITY;
+      if (fast) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NT; ++j)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int key = c0 + 8 * j + 2 * qd + e;
-          float v = -INFINITY;
-          if (j < ntc && row_on && key < rows) {
-            const float Sv = s[j][e] * a.qscale;
-            if (tok0 + key == a.n - 1) {
-              v = Sv * kLog2e;  // the current token is exempt from the gate
-            } else {
-              const float x = a.beta * (Sv - tau_r);
-              v = Sv * rcp_approx(1.0f + ex2_approx(-x * kLog2e)) * kLog2e;
-            }
+          for (int e = 0; e < 2; ++e) {
+            const float v = row_on ? gate((se[j][e] + so[j][e]) * a.qscale) : -INFINITY;
+            g[j][e] = v;
+            bm = fmaxf(bm, v);
           }
-          g[j][e] = v;
-          bm = fmaxf(bm, v);
-        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int key = c0 + 8 * j + 2 * qd + e;
+            float v = -INFINITY;
+            if (row_on && key < rows) {
+              const float Sv = (se[j][e] + so[j][e]) * a.qscale;
+              // the current token is exempt from the gate (Eq. 3)
+              v = (tok0 + key == a.n - 1) ? Sv * kLog2e : gate(Sv);
+            }
+            g[j][e] = v;
+            bm = fmaxf(bm, v);
+          }
+      }
       bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 1));
       bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 2));
       const float mn = fmaxf(m_r, bm);
       float corr = 1.0f, ps = 0.0f;
-      float p[4][2];
+      float p[NT][2];
       if (mn != -INFINITY) {
         corr = ex2_approx(m_r - mn);
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
+        for (int j = 0; j < NT; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             p[j][e] = ex2_approx(g[j][e] - mn);
@@ -301,7 +317,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           }
       } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) p[j][0] = p[j][1] = 0.0f;
+        for (int j = 0; j < NT; ++j) p[j][0] = p[j][1] = 0.0f;
       }
       l_r = fmaf(l_r, corr, ps);
       m_r = mn;
@@ -314,26 +330,23 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
           o[j][3] *= corr;
         }
       }
-      // O += P V, P = hi + lo in bf16
+      // O += P V, P = high + low parts in bf16
 #pragma unroll
-      for (int m2 = 0; m2 < 2; ++m2) {
-        if (2 * m2 < ntc) {
-          const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
-          const uint32_t h1 = pack_bf16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
-          const __nv_bfloat162 hb0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
-          const __nv_bfloat162 hb1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
-          const uint32_t l0 = pack_bf16x2(p[2 * m2][0] - __low2float(hb0), p[2 * m2][1] - __high2float(hb0));
-          const uint32_t l1 =
-              pack_bf16x2(p[2 * m2 + 1][0] - __low2float(hb1), p[2 * m2 + 1][1] - __high2float(hb1));
-          const int vrow = c0 + 16 * m2 + 8 * ((lane >> 3) & 1) + (lane & 7);
+      for (int m2 = 0; m2 < NT / 2; ++m2) {
+        const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
+        const uint32_t h1 = pack_bf16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
+        const __nv_bfloat162 hb0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
+        const __nv_bfloat162 hb1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
+        const uint32_t l0 = pack_bf16x2(p[2 * m2][0] - __low2float(hb0), p[2 * m2][1] - __high2float(hb0));
+        const uint32_t l1 = pack_bf16x2(p[2 * m2 + 1][0] - __low2float(hb1), p[2 * m2 + 1][1] - __high2float(hb1));
+        const int vrow = c0 + 16 * m2 + 8 * ((lane >> 3) & 1) + (lane & 7);
 #pragma unroll
-          for (int jd = 0; jd < NDT; jd += 2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
-            // A rows 0-7: high part, rows 8-15: low part of the same P row
-            mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
-            mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
-          }
+        for (int jd = 0; jd < NDT; jd += 2) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
+          // A rows 0-7: high part, rows 8-15: low part of the same P row
+          mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
+          mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
         }
       }
     }
@@ -395,7 +408,7 @@ bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int b
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G, bool DENSE>
+template <int D, int G, bool DENSE, int CH>
 cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
@@ -417,29 +430,35 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
     return cudaErrorInvalidValue;
 
   static std::atomic<uint64_t> smem_done{0};
-  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE>));
+  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH>));
   if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(c, nst);
-  decode_mma_kernel<D, G, DENSE><<<c.S, kMmaThreads, smem, st>>>(a, tmk, tmv);
+  decode_mma_kernel<D, G, DENSE, CH><<<c.S, kMmaThreads, smem, st>>>(a, tmk, tmv);
   return cudaGetLastError();
 }
 
-template <int D, bool DENSE>
+template <int D, bool DENSE, int CH>
 cudaError_t launch_mma_g(const DecodeCall& c, cudaStream_t st) {
   switch (c.shape.n_q_heads / c.shape.n_kv_heads) {
-    case 1: return launch_mma_t<D, 1, DENSE>(c, st);
-    case 2: return launch_mma_t<D, 2, DENSE>(c, st);
-    case 4: return launch_mma_t<D, 4, DENSE>(c, st);
-    case 8: return launch_mma_t<D, 8, DENSE>(c, st);
+    case 1: return launch_mma_t<D, 1, DENSE, CH>(c, st);
+    case 2: return launch_mma_t<D, 2, DENSE, CH>(c, st);
+    case 4: return launch_mma_t<D, 4, DENSE, CH>(c, st);
+    case 8: return launch_mma_t<D, 8, DENSE, CH>(c, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Chunks of 32 keys, or 16 for 16-token blocks.
+template <int D, bool DENSE>
+cudaError_t launch_mma_c(const DecodeCall& c, cudaStream_t st) {
+  return c.shape.block_size == 16 ? launch_mma_g<D, DENSE, 16>(c, st) : launch_mma_g<D, DENSE, 32>(c, st);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_mma(const DecodeCall& c, cudaStream_t st) {
-  if (c.shape.head_dim == 128) return c.dense ? launch_mma_g<128, true>(c, st) : launch_mma_g<128, false>(c, st);
-  return c.dense ? launch_mma_g<64, true>(c, st) : launch_mma_g<64, false>(c, st);
+  if (c.shape.head_dim == 128) return c.dense ? launch_mma_c<128, true>(c, st) : launch_mma_c<128, false>(c, st);
+  return c.dense ? launch_mma_c<64, true>(c, st) : launch_mma_c<64, false>(c, st);
 }
 
 }  // namespace eta
