@@ -222,6 +222,32 @@ ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params
                                       int64_t tau_batch_stride, float* out, void* workspace, size_t ws_bytes,
                                       eta_stream_t stream);
 
+/*
+ * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and
+ * without any device allocation. The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory when they
+ * decode (a CUDA graph being captured, a serving engine whose memory plan is
+ * frozen at start-up, a host framework that owns every allocation, a
+ * real-time loop that must not enter an allocator).
+ *
+ * The scratch is a fixed array of ETA_STATIC_SCRATCH_BYTES inside the library,
+ * one per device that loads it, held until the process exits. Shapes whose
+ * eta_decode_workspace_bytes exceeds that size are rejected with
+ * ETA_ERR_WORKSPACE before anything is launched. All calls on a device share
+ * the array: calls whose kernels overlap on the GPU (unordered streams) race
+ * and must not be issued. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress); make it before any stream capture.
+ * Each call clears the scratch status word first. device_status (nullable,
+ * device memory) receives this call's device status word, stream-ordered.
+ * Other arguments and results as eta_decode_sparse.
+ */
+#define ETA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+ETA_API eta_status_t eta_decode_sparse_static(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                              const void* k, const void* v, eta_meta_t meta, int64_t n_tokens,
+                                              const float* tau, int64_t tau_batch_stride, float* out,
+                                              const eta_screen_out_t* extra, int32_t* device_status,
+                                              eta_stream_t stream);
+
 /* Synchronise `stream`, read the workspace's device status word into *status
  * (host pointer) and clear it. Returns ETA_ERR_CUDA if the copy fails. */
 ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t stream, eta_status_t* status);

@@ -74,6 +74,9 @@ def _load():
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
     L.eta_decode_dense.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
+    L.eta_decode_sparse_static.restype = st
+    L.eta_decode_sparse_static.argtypes = [P(Shape), P(Params), vp, vp, vp, Meta, i64, vp, i64, vp, P(ScreenOut),
+                                           vp, vp]
     L.eta_read_device_status.restype = st
     L.eta_read_device_status.argtypes = [vp, vp, P(st)]
     return L
@@ -82,7 +85,8 @@ def _load():
 lib = _load()
 EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta_predict_tau",
             "eta_decode_workspace_bytes", "eta_workspace_init", "eta_screen", "eta_decode_sparse",
-            "eta_decode_screened", "eta_decode_dense", "eta_read_device_status")
+            "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static")
+STATIC_SCRATCH_BYTES = 32 << 20
 
 
 def status_string(status: int) -> str:
@@ -186,6 +190,18 @@ def decode_dense(shape: Shape, params: Params, q, k, v, n_tokens: int, tau: Opti
     _check(lib.eta_decode_dense(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), n_tokens,
                                 _ptr(tau), tau_batch_stride, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "eta_decode_dense")
+
+
+def decode_sparse_static(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, tau: torch.Tensor,
+                         tau_batch_stride: int, out: torch.Tensor, device_status: Optional[torch.Tensor] = None,
+                         stream=None, **outs) -> None:
+    """eta_decode_sparse on the library's fixed device scratch: no workspace and
+    no allocation (for callers that cannot allocate while decoding)."""
+    so = _screen_out(**outs)
+    _check(lib.eta_decode_sparse_static(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                        Meta(*(m.data_ptr() for m in meta)), n_tokens, _ptr(tau), tau_batch_stride,
+                                        _ptr(out), ctypes.byref(so) if so is not None else None,
+                                        _ptr(device_status), _stream(stream)), "eta_decode_sparse_static")
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:
