@@ -237,6 +237,10 @@ ETA_API eta_status_t eta_predict_tau(const eta_shape_t* shape, const void* q, co
   if (q == nullptr || W == nullptr || bias == nullptr || tau == nullptr) return ETA_ERR_INVALID_ARG;
   if (!aligned(q, elem_bytes(shape->q_dtype)) || !aligned(W, 4) || !aligned(bias, 4) || !aligned(tau, 4))
     return ETA_ERR_INVALID_ARG;
+  // the kernel stages one batch row of queries (Hq*d fp32) in shared memory
+  if (static_cast<size_t>(shape->n_q_heads) * shape->head_dim * 4 + 8192 >
+      static_cast<size_t>(device_max_smem_optin()))
+    return ETA_ERR_UNSUPPORTED;
   return from_cuda(launch_predict(*shape, q, W, bias, tau, stream));
 }
 

@@ -3,9 +3,10 @@
 //
 // One thread-block cluster per (batch, kv head). Each CTA of the cluster scores
 // a contiguous range of 32-block tiles, one warp lane per block and all G query
-// heads of the GQA group at once (the metadata is read once per group). The
-// metadata is coordinate-major, so for every coordinate i a warp reads 128
-// contiguous bytes of mu and of var. Per-tile admission counts give the CTA's
+// heads of the GQA group at once (the metadata is read once per group). A warp
+// scores 4 consecutive tiles together: the metadata is coordinate-major, so
+// for every coordinate i it reads 512 contiguous bytes of mu and of var, with
+// the loads of several coordinates in flight. Per-tile admission counts give the CTA's
 // local offsets; the CTAs exchange their totals through distributed shared
 // memory, so the cluster writes one globally ascending list without another
 // launch. The union over the group (the blocks that must be loaded, with a
@@ -21,7 +22,8 @@ namespace eta {
 
 namespace {
 
-constexpr int kScreenWarps = 8;
+constexpr int kScreenWarps = 4;
+constexpr int kSub = 4;  // tiles a warp scores together
 
 struct ScreenArgs {
   const void* q;
@@ -92,42 +94,63 @@ __global__ void __launch_bounds__(kScreenWarps * 32) screen_kernel(const ScreenA
   const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
 
   // Phase 1: score and decide every screened block of this CTA's tiles.
-  for (int t = warp; t < my_tiles; t += kScreenWarps) {
-    const int blk = (t0 + t) * 32 + lane;
-    const bool valid = blk < a.ns;
-    const int cb = valid ? blk : a.ns - 1;
-    float dg[G], vg[G];
+  for (int t4 = warp * kSub; t4 < my_tiles; t4 += kScreenWarps * kSub) {
+    int cb[kSub];
+    bool valid[kSub];
 #pragma unroll
-    for (int g = 0; g < G; ++g) dg[g] = vg[g] = 0.0f;
+    for (int u = 0; u < kSub; ++u) {
+      const int blk = (t0 + t4 + u) * 32 + lane;
+      valid[u] = (t4 + u < my_tiles) && blk < a.ns;
+      cb[u] = blk < a.ns ? blk : a.ns - 1;
+    }
+    float dg[kSub][G], vg[kSub][G];
+#pragma unroll
+    for (int u = 0; u < kSub; ++u)
+#pragma unroll
+      for (int g = 0; g < G; ++g) dg[u][g] = vg[u][g] = 0.0f;
 #pragma unroll 8
     for (int i = 0; i < D; ++i) {
-      const float m = __ldg(mu + static_cast<int64_t>(i) * a.nb_cap + cb);
-      const float v = __ldg(var + static_cast<int64_t>(i) * a.nb_cap + cb);
+      float m[kSub], v[kSub];
+#pragma unroll
+      for (int u = 0; u < kSub; ++u) {
+        m[u] = __ldg(mu + static_cast<int64_t>(i) * a.nb_cap + cb[u]);
+        v[u] = __ldg(var + static_cast<int64_t>(i) * a.nb_cap + cb[u]);
+      }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        dg[g] = __fmaf_rn(s_q[g * D + i], m, dg[g]);
-        vg[g] = __fmaf_rn(s_qq[g * D + i], v, vg[g]);
+        const float qi = s_q[g * D + i], qqi = s_qq[g * D + i];
+#pragma unroll
+        for (int u = 0; u < kSub; ++u) {
+          dg[u][g] = __fmaf_rn(qi, m[u], dg[u][g]);
+          vg[u][g] = __fmaf_rn(qqi, v[u], vg[u][g]);
+        }
       }
     }
-    const float M = __ldg(mx + cb);
-    uint32_t mask = 0;
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float A = __fadd_rn(dg[g], __fmul_rn(a.z, __fsqrt_rn(vg[g])));
-      const float C = __fmul_rn(s_qn[g], M);
-      const float sc = __fmul_rn((A < C) ? A : C, a.s);
-      if (valid && !(sc < s_taut[g])) mask |= 1u << g;
-      if (a.scores != nullptr && valid)
-        a.scores[(static_cast<int64_t>(b) * a.Hq + kvh * G + g) * a.nb_cap + blk] = sc;
-    }
-    s_mask[t * 32 + lane] = static_cast<uint8_t>(mask);
-    int cnt[G + 1];
+    for (int u = 0; u < kSub; ++u) {
+      if (t4 + u >= my_tiles) break;  // uniform over the warp
+      const int t = t4 + u;
+      const int blk = (t0 + t) * 32 + lane;
+      const float M = __ldg(mx + cb[u]);
+      uint32_t mask = 0;
 #pragma unroll
-    for (int g = 0; g < G; ++g) cnt[g] = __popc(__ballot_sync(kFull, (mask >> g) & 1u));
-    cnt[G] = __popc(__ballot_sync(kFull, mask != 0u));
-    if (lane == 0) {
+      for (int g = 0; g < G; ++g) {
+        const float A = __fadd_rn(dg[u][g], __fmul_rn(a.z, __fsqrt_rn(vg[u][g])));
+        const float C = __fmul_rn(s_qn[g], M);
+        const float sc = __fmul_rn((A < C) ? A : C, a.s);
+        if (valid[u] && !(sc < s_taut[g])) mask |= 1u << g;
+        if (a.scores != nullptr && valid[u])
+          a.scores[(static_cast<int64_t>(b) * a.Hq + kvh * G + g) * a.nb_cap + blk] = sc;
+      }
+      s_mask[t * 32 + lane] = static_cast<uint8_t>(mask);
+      int cnt[G + 1];
 #pragma unroll
-      for (int c = 0; c <= G; ++c) s_tcnt[t * (G + 1) + c] = cnt[c];
+      for (int g = 0; g < G; ++g) cnt[g] = __popc(__ballot_sync(kFull, (mask >> g) & 1u));
+      cnt[G] = __popc(__ballot_sync(kFull, mask != 0u));
+      if (lane == 0) {
+#pragma unroll
+        for (int c = 0; c <= G; ++c) s_tcnt[t * (G + 1) + c] = cnt[c];
+      }
     }
   }
   __syncthreads();
@@ -213,10 +236,9 @@ cudaError_t launch_screen_t(const ScreenCall& c, cudaStream_t st) {
   const int nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
   const int ns = max(0, nb - c.n_local);
   const int nt = (ns + 31) / 32;
-  // Enough CTAs to cover the SMs about twice, at most kMaxCluster per cluster.
-  int cs = (2 * device_sm_count() + BH - 1) / BH;
-  cs = max(1, min(cs, kMaxCluster));
-  cs = max(1, min(cs, nt));
+  // As many CTAs per cluster as there are tiles, up to kMaxCluster: the tiles
+  // of a (batch, kv head) spread evenly, each warp scoring kSub at a time.
+  int cs = max(1, min(kMaxCluster, nt));
   while ((nt + cs - 1) / cs > kMaxScreenTiles && cs < kMaxCluster) ++cs;
   const int tpc = max(1, (nt + cs - 1) / cs);
   if (tpc > kMaxScreenTiles) return cudaErrorInvalidValue;
