@@ -80,13 +80,45 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Largest value over the ranks (device time of the slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(queries_per_rank: int, ms_max: float, world: int) -> float:
+    """Whole-job queries/s: every rank decodes its own batch (weak scaling); the
+    job takes as long as its slowest rank."""
+    return world * queries_per_rank / (ms_max * 1e-3)
+
+
+def decode_sources_digest() -> str:
+    """sha256 over the sources that define the tensor-core decode kernel."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("decode_mma.cu", "decode_common.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "learned_block_sparse_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload_name: str, union_blocks: int):
+    """DRAM bytes per decode launch from the committed ncu capture
+    (profiles/decode_traffic.json), scaled by admitted union blocks; None when
+    the capture is missing, is for another workload, or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    if d.get("source_sha256") != decode_sources_digest() or d.get("workload") != workload_name:
+        return None
+    return float(d["dram_bytes_per_union_block"]) * union_blocks
 
 
 def measured_peaks():
@@ -411,7 +443,7 @@ def run_eta(args):
     ms = max_over_ranks(main["ms"], world)
     ms_dec = max_over_ranks(main["ms_decode"], world)
     queries = w.B * w.Hq
-    value = world * queries / (ms * 1e-3)
+    value = job_throughput(queries, ms, world)
     bm = main["bytes"]
     peak, peak_kind = measured_peaks()
     achieved = bm["decode_kernel"] / (ms_dec * 1e-3) / 1e9
@@ -424,12 +456,12 @@ def run_eta(args):
                    "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
                    "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
         "effective_hbm_gbs": bm["step_read"] / (ms * 1e-3) / 1e9,
-        "d_head": bm["d_head"], "d_union": bm["d_union"],
+        "d_head": bm["d_head"], "d_union": bm["d_union"], "union_blocks": bm["union_blocks"],
         "phases_ms": {"predict": main["ms_predict"], "screen": main["ms_screen"],
                       "decode_combine": main["ms_decode"]},
         "roofline": {"bound": "hbm", "kernel": "decode_kernel (+combine, timed together)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": peak_kind, "traffic": None,
+                     "peak_source": peak_kind, "traffic": measured_traffic(w.name, bm["union_blocks"]),
                      "bytes_per_launch": bm["decode_kernel"]},
         "gpu_launches": LAUNCHES_PER_STEP[w.tau_mode] * args.steps,
         "clocks": main["clocks"],
