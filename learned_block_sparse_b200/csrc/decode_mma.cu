@@ -375,7 +375,15 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     if (finished || p >= hi) break;
     const int it = static_cast<int>(p - lo);
     const int st = it % NST;
-    const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, a.status);
+    const int round = it / NST;
+    // Consecutive uses of a stage belong to different warps, so this warp may
+    // get here before the stage's previous use has even landed; an mbarrier
+    // wait on a phase two ahead of the current one would return at once. Wait
+    // for the previous use's release first: then the full barrier is at most
+    // one phase behind and the parity wait below is exact.
+    bool ok = round == 0 || mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>((round - 1) & 1), s_abort,
+                                              a.status);
+    ok = ok && mbar_wait_bounded(&s_full[st], static_cast<uint32_t>(round & 1), s_abort, a.status);
     if (ok) process(st, s_info[st]);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s_empty[st]);

@@ -131,6 +131,15 @@ def test_dtypes_dims_blocks(dtype, d, bs):
     _full_check(w, dense=True)
 
 
+@pytest.mark.parametrize("bs,n_splits", [(64, 2), (64, 5), (128, 3), (32, 4), (16, 3)])
+def test_long_ranges_reuse_every_stage_many_times(bs, n_splits):
+    """Few split ranges, so each thread block streams hundreds of blocks through
+    its ring and every stage is reused many times by different consumer warps."""
+    w = synth.Workload("ring", "bf16", 1, 4, 4, 128, bs * 700 + 3, bs, z=1.0, tau_mode="const",
+                       densities=(0.5,), seed=bs + n_splits, offset_std=synth.SQRT_HALF)
+    _full_check(w, 0.5, n_splits=n_splits, dense=True)
+
+
 def test_edge_single_token_and_exact_blocks():
     for n in (1, 16, 17, 32):
         w = synth.Workload("e", "bf16", 1, 2, 2, 128, n, 16, z=1.0, tau_mode="const", densities=(0.5,), seed=n,
