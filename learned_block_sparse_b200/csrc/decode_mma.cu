@@ -381,8 +381,10 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     // wait on a phase two ahead of the current one would return at once. Wait
     // for the previous use's release first: then the full barrier is at most
     // one phase behind and the parity wait below is exact.
-    bool ok = round == 0 || mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>((round - 1) & 1), s_abort,
-                                              a.status);
+    // (With a stage count that is a multiple of kMW a stage always returns to
+    // the same warp, which has released it itself, and the extra wait is skipped.)
+    bool ok = round == 0 || (NST % kMW) == 0 ||
+              mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>((round - 1) & 1), s_abort, a.status);
     ok = ok && mbar_wait_bounded(&s_full[st], static_cast<uint32_t>(round & 1), s_abort, a.status);
     if (ok) process(st, s_info[st]);
     __syncwarp();
@@ -430,6 +432,9 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const size_t nst_bw = (200 * 1024) / (2 * tile), nst_fit = (budget - fixed) / per_stage;
   int nst = static_cast<int>(nst_bw < nst_fit ? nst_bw : nst_fit);
   nst = max(2, min(nst, 24));
+  // With at least 2*kMW stages, round down to a multiple of kMW so a stage
+  // always returns to the warp that released it (see the consumer loop).
+  if (nst >= 2 * kMW) nst -= nst % kMW;
   const size_t smem = static_cast<size_t>(nst) * per_stage + fixed + 64;
 
   CUtensorMap tmk, tmv;

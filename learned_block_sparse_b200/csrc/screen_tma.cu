@@ -1,0 +1,226 @@
+// Block screening (Methodology §4, Eq. 5 and the admission rule) with the
+// metadata tiles staged by TMA.
+//
+// Same cluster layout and compaction as screen.cu (one cluster per (batch, kv
+// head), lane = block, all G heads of the group per metadata read). Here a
+// producer warp streams each 32-block tile's metadata, one 2-D box of
+// [d coordinates][32 blocks] of mu and one of var (32 KB at d = 128), into a
+// ring of shared-memory stages; consumer warp w scores tiles w, w + CW, ... from
+// shared memory (lane = column, so the reads are conflict-free) with the
+// multiply-adds in increasing coordinate order. The ring keeps several tiles in
+// flight per SM even when a (batch, kv head) has few tiles, which plain loads
+// from a handful of warps cannot. The stage count is a multiple of the consumer
+// count, so a stage always returns to the warp that released it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "screen_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace eta {
+
+namespace {
+
+template <int D> struct TmaScreenCfg;
+template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 6; };
+template <> struct TmaScreenCfg<64> { static constexpr int kCW = 4, kNST = 12; };
+
+__device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(tm), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 1)
+    screen_tma_kernel(const ScreenArgs a, int32_t* status, const __grid_constant__ CUtensorMap tmu,
+                      const __grid_constant__ CUtensorMap tvar) {
+  constexpr int CW = TmaScreenCfg<D>::kCW;
+  constexpr int NST = TmaScreenCfg<D>::kNST;
+  constexpr int NT = (CW + 1) * 32;
+  constexpr uint32_t kBox = D * 32 * sizeof(float);  // one array's tile
+  static_assert(NST % CW == 0, "stages must return to the same consumer warp");
+  cg::cluster_group cluster = cg::this_cluster();
+  const int cs = static_cast<int>(cluster.num_blocks());
+  const int cr = static_cast<int>(cluster.block_rank());
+  const int bh = blockIdx.x / cs;
+  const int b = bh / a.Hkv, kvh = bh % a.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tpc = a.tiles_per_cta;
+
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  unsigned char* smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);
+  float* s_stage = reinterpret_cast<float*>(smem);  // [NST][2][D][32]
+  uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * kBox);
+  uint64_t* s_empty = s_full + NST;
+  int* s_abort = reinterpret_cast<int*>(s_empty + NST);
+  const ScreenSmem<D, G> sm(reinterpret_cast<unsigned char*>(s_abort + 4), tpc);
+
+  if (tid == 0) {
+    *s_abort = 0;
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  screen_prologue<D, G>(a, sm, b, kvh, NT);  // ends with __syncthreads
+
+  const int nt = (a.ns + 31) / 32;
+  const int t0 = cr * tpc;
+  const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
+  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
+
+  if (warp == CW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      bool aborted = false;
+      for (int it = 0; it < my_tiles && !aborted; ++it) {
+        const int st = it % NST, round = it / NST;
+        if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status)) {
+          aborted = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&s_full[st], 2 * kBox);
+        const int x = (t0 + it) * 32, y = bh * D;
+        tma_load_2d_plain(s_stage + static_cast<size_t>(st) * 2 * D * 32, &tmu, x, y, &s_full[st]);
+        tma_load_2d_plain(s_stage + (static_cast<size_t>(st) * 2 + 1) * D * 32, &tvar, x, y, &s_full[st]);
+        issued = it + 1;
+      }
+      if (aborted) {  // let the copies already issued land before exiting
+        for (int j = max(0, issued - NST); j < issued; ++j) {
+          const uint64_t tstart = global_timer_ns();
+          while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - tstart < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    for (int it = warp; it < my_tiles; it += CW) {
+      const int st = it % NST;
+      const int blk = (t0 + it) * 32 + lane;
+      const bool valid = blk < a.ns;
+      const float M = __ldg(mx + (valid ? blk : a.ns - 1));
+      const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status);
+      float dg[G], vg[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) dg[g] = vg[g] = 0.0f;
+      if (ok) {
+        const float* mu_s = s_stage + static_cast<size_t>(st) * 2 * D * 32;
+        const float* var_s = mu_s + D * 32;
+#pragma unroll 8
+        for (int i = 0; i < D; ++i) {
+          const float m = mu_s[i * 32 + lane], v = var_s[i * 32 + lane];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            dg[g] = __fmaf_rn(sm.q[g * D + i], m, dg[g]);
+            vg[g] = __fmaf_rn(sm.qq[g * D + i], v, vg[g]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[st]);
+      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, blk, valid, dg, vg, M));
+    }
+  }
+  __syncthreads();
+  screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, NT);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 meta_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows][nb_cap] fp32 view of mu or var, boxes of [d rows][32 blocks].
+bool encode_meta_map(CUtensorMap* tm, const float* base, int64_t rows, int64_t nb_cap, int d) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = meta_map_encoder();
+  if (enc == nullptr) return false;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(nb_cap), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(nb_cap) * sizeof(float)};
+  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(d)};
+  const cuuint32_t estride[2] = {1u, 1u};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G>
+cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
+  constexpr int CW = TmaScreenCfg<D>::kCW, NST = TmaScreenCfg<D>::kNST;
+  const eta_shape_t& s = c.shape;
+  const int BH = s.batch * s.n_kv_heads;
+  const int64_t nb_cap = s.capacity / s.block_size;
+  const int nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
+  const int ns = max(0, nb - c.n_local);
+  const int nt = (ns + 31) / 32;
+  const int cs = max(1, min(kMaxCluster, nt));
+  const int tpc = max(1, (nt + cs - 1) / cs);
+  if (tpc > kMaxScreenTiles) return cudaErrorInvalidValue;
+  const size_t smem = 128 + static_cast<size_t>(NST) * 2 * D * 32 * sizeof(float) + 2 * NST * sizeof(uint64_t) +
+                      4 * sizeof(int) + ScreenSmem<D, G>::bytes(tpc);
+  if (smem > static_cast<size_t>(device_max_smem_optin())) return cudaErrorNotSupported;
+  CUtensorMap tmu, tvar;
+  const int64_t rows = static_cast<int64_t>(BH) * D;
+  if (!encode_meta_map(&tmu, c.meta.mu, rows, nb_cap, D) || !encode_meta_map(&tvar, c.meta.var, rows, nb_cap, D))
+    return cudaErrorNotSupported;
+  const ScreenArgs a = make_screen_args(c, nb, ns, tpc);
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(screen_tma_kernel<D, G>));
+  if (e != cudaSuccess) return e;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(BH * cs));
+  cfg.blockDim = dim3((CW + 1) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, screen_tma_kernel<D, G>, a, c.ws.status, tmu, tvar);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_tma_d(const ScreenCall& c, cudaStream_t st) {
+  switch (c.shape.n_q_heads / c.shape.n_kv_heads) {
+    case 1: return launch_tma_t<D, 1>(c, st);
+    case 2: return launch_tma_t<D, 2>(c, st);
+    case 4: return launch_tma_t<D, 4>(c, st);
+    case 8: return launch_tma_t<D, 8>(c, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_screen_tma(const ScreenCall& c, cudaStream_t st) {
+  const int64_t nb_cap = c.shape.capacity / c.shape.block_size;
+  // TMA wants 16-byte aligned rows and a 16-byte aligned base
+  if (nb_cap % 4 != 0 || (reinterpret_cast<uintptr_t>(c.meta.mu) & 15) != 0 ||
+      (reinterpret_cast<uintptr_t>(c.meta.var) & 15) != 0)
+    return cudaErrorNotSupported;
+  return c.shape.head_dim == 128 ? launch_tma_d<128>(c, st) : launch_tma_d<64>(c, st);
+}
+
+}  // namespace eta

@@ -93,12 +93,14 @@ class Workload:
     offset_std: float = 0.0
     n_needles: int = 0
     needle_scale: float = 3.0
-    cap: Optional[int] = None    # allocated tokens per (b, kv head); default n rounded up to bs
+    cap: Optional[int] = None    # allocated tokens per (b, kv head); default n rounded up to 4 blocks
 
     @property
     def capacity(self) -> int:
-        c = self.cap if self.cap is not None else self.n
-        return ((c + self.bs - 1) // self.bs) * self.bs
+        if self.cap is not None:
+            return ((self.cap + self.bs - 1) // self.bs) * self.bs
+        q = 4 * self.bs          # whole groups of 4 blocks: 16-byte aligned metadata rows
+        return ((self.n + q - 1) // q) * q
 
     @property
     def nb(self) -> int:

@@ -140,6 +140,16 @@ def test_long_ranges_reuse_every_stage_many_times(bs, n_splits):
     _full_check(w, 0.5, n_splits=n_splits, dense=True)
 
 
+@pytest.mark.parametrize("cfg,blocks", [(3, 151), (5, 301), (2, 41)])
+def test_screen_plain_loads_when_metadata_rows_unaligned(cfg, blocks):
+    """capacity / block_size not a multiple of 4: metadata rows are not 16-byte
+    aligned, so the screen takes the plain-load kernel instead of TMA staging."""
+    w = _reduced(cfg)
+    w = w.replace(cap=blocks * w.bs)
+    assert (w.capacity // w.bs) % 4 != 0
+    _full_check(w, w.densities[0])
+
+
 def test_edge_single_token_and_exact_blocks():
     for n in (1, 16, 17, 32):
         w = synth.Workload("e", "bf16", 1, 2, 2, 128, n, 16, z=1.0, tau_mode="const", densities=(0.5,), seed=n,
