@@ -216,6 +216,13 @@ cudaError_t launch_tma_d(const ScreenCall& c, cudaStream_t st) {
 
 cudaError_t launch_screen_tma(const ScreenCall& c, cudaStream_t st) {
   const int64_t nb_cap = c.shape.capacity / c.shape.block_size;
+  // Staging pays off while the launch is latency bound: fewer thread blocks
+  // than about two per SM. Larger launches keep enough plain loads in flight
+  // (several blocks per SM), while the ring's shared memory allows one.
+  const int nb = static_cast<int>((c.n + c.shape.block_size - 1) / c.shape.block_size);
+  const int nt = (max(0, nb - c.n_local) + 31) / 32;
+  const int64_t ctas = static_cast<int64_t>(c.shape.batch) * c.shape.n_kv_heads * max(1, min(kMaxCluster, nt));
+  if (ctas >= 2 * static_cast<int64_t>(device_sm_count())) return cudaErrorNotSupported;
   // TMA wants 16-byte aligned rows and a 16-byte aligned base
   if (nb_cap % 4 != 0 || (reinterpret_cast<uintptr_t>(c.meta.mu) & 15) != 0 ||
       (reinterpret_cast<uintptr_t>(c.meta.var) & 15) != 0)
