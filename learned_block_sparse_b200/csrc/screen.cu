@@ -25,7 +25,7 @@ constexpr int kScreenWarps = 4;
 constexpr int kSub = 4;  // tiles a warp scores together
 
 template <int D, int G>
-__global__ void __launch_bounds__(kScreenWarps * 32) screen_kernel(const ScreenArgs a) {
+__global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const ScreenArgs a) {
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
