@@ -79,8 +79,14 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
   }
   __syncthreads();
   if (tid < G) {
-    float qn = 0.0f;
-    for (int e = 0; e < D; ++e) qn = __fmaf_rn(sm.q[tid * D + e], sm.q[tid * D + e], qn);
+    float qn = 0.0f;  // sum of q_i^2 by fused multiply-adds in increasing i
+    for (int e0 = 0; e0 < D; e0 += 16) {
+      float x[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) x[c] = sm.q[tid * D + e0 + c];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) qn = __fmaf_rn(x[c], x[c], qn);
+    }
     sm.qn[tid] = __fsqrt_rn(qn);
     sm.taut[tid] = __fsub_rn(a.tau[b * a.tau_stride + kvh * G + tid], a.offset_a);
   }

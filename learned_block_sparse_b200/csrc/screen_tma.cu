@@ -25,8 +25,9 @@ namespace eta {
 namespace {
 
 template <int D> struct TmaScreenCfg;
-template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 6; };
-template <> struct TmaScreenCfg<64> { static constexpr int kCW = 4, kNST = 12; };
+// 96 KB of stages: two thread blocks per SM.
+template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 3; };
+template <> struct TmaScreenCfg<64> { static constexpr int kCW = 3, kNST = 6; };
 
 __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -37,7 +38,7 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 1)
+__global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
     screen_tma_kernel(const ScreenArgs a, int32_t* status, const __grid_constant__ CUtensorMap tmu,
                       const __grid_constant__ CUtensorMap tvar) {
   constexpr int CW = TmaScreenCfg<D>::kCW;
@@ -61,6 +62,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 1)
   int* s_abort = reinterpret_cast<int*>(s_empty + NST);
   const ScreenSmem<D, G> sm(reinterpret_cast<unsigned char*>(s_abort + 4), tpc);
 
+  const int nt = (a.ns + 31) / 32;
+  const int t0 = cr * tpc;
+  const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
+  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
+
   if (tid == 0) {
     *s_abort = 0;
     for (int s = 0; s < NST; ++s) {
@@ -69,28 +75,32 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 1)
     }
     fence_mbar_init();
   }
+  __syncthreads();
+  auto issue_tile = [&](int it) {
+    const int st = it % NST;
+    mbar_arrive_expect_tx(&s_full[st], 2 * kBox);
+    const int x = (t0 + it) * 32, y = bh * D;
+    tma_load_2d_plain(s_stage + static_cast<size_t>(st) * 2 * D * 32, &tmu, x, y, &s_full[st]);
+    tma_load_2d_plain(s_stage + (static_cast<size_t>(st) * 2 + 1) * D * 32, &tvar, x, y, &s_full[st]);
+  };
+  // the first ring of tiles does not depend on the queries: start it now
+  const int first = my_tiles < NST ? my_tiles : NST;
+  if (warp == CW && lane == 0)
+    for (int it = 0; it < first; ++it) issue_tile(it);
   screen_prologue<D, G>(a, sm, b, kvh, NT);  // ends with __syncthreads
-
-  const int nt = (a.ns + 31) / 32;
-  const int t0 = cr * tpc;
-  const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
-  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0;
+      int issued = first;
       bool aborted = false;
-      for (int it = 0; it < my_tiles && !aborted; ++it) {
+      for (int it = first; it < my_tiles && !aborted; ++it) {
         const int st = it % NST, round = it / NST;
-        if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status)) {
+        if (!mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status)) {
           aborted = true;
           break;
         }
-        mbar_arrive_expect_tx(&s_full[st], 2 * kBox);
-        const int x = (t0 + it) * 32, y = bh * D;
-        tma_load_2d_plain(s_stage + static_cast<size_t>(st) * 2 * D * 32, &tmu, x, y, &s_full[st]);
-        tma_load_2d_plain(s_stage + (static_cast<size_t>(st) * 2 + 1) * D * 32, &tvar, x, y, &s_full[st]);
+        issue_tile(it);
         issued = it + 1;
       }
       if (aborted) {  // let the copies already issued land before exiting
@@ -115,13 +125,27 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 1)
       if (ok) {
         const float* mu_s = s_stage + static_cast<size_t>(st) * 2 * D * 32;
         const float* var_s = mu_s + D * 32;
-#pragma unroll 8
-        for (int i = 0; i < D; ++i) {
-          const float m = mu_s[i * 32 + lane], v = var_s[i * 32 + lane];
+#pragma unroll 2
+        for (int i0 = 0; i0 < D; i0 += 4) {
+          float m[4], v[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            m[c] = mu_s[(i0 + c) * 32 + lane];
+            v[c] = var_s[(i0 + c) * 32 + lane];
+          }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            dg[g] = __fmaf_rn(sm.q[g * D + i], m, dg[g]);
-            vg[g] = __fmaf_rn(sm.qq[g * D + i], v, vg[g]);
+            // four coordinates of q and q*q per shared load; multiply-adds in coordinate order
+            const float4 qv = *reinterpret_cast<const float4*>(sm.q + g * D + i0);
+            const float4 qqv = *reinterpret_cast<const float4*>(sm.qq + g * D + i0);
+            dg[g] = __fmaf_rn(qv.x, m[0], dg[g]);
+            dg[g] = __fmaf_rn(qv.y, m[1], dg[g]);
+            dg[g] = __fmaf_rn(qv.z, m[2], dg[g]);
+            dg[g] = __fmaf_rn(qv.w, m[3], dg[g]);
+            vg[g] = __fmaf_rn(qqv.x, v[0], vg[g]);
+            vg[g] = __fmaf_rn(qqv.y, v[1], vg[g]);
+            vg[g] = __fmaf_rn(qqv.z, v[2], vg[g]);
+            vg[g] = __fmaf_rn(qqv.w, v[3], vg[g]);
           }
         }
       }
@@ -169,7 +193,11 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   const int nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
   const int ns = max(0, nb - c.n_local);
   const int nt = (ns + 31) / 32;
-  const int cs = max(1, min(kMaxCluster, nt));
+  // Clusters as large as keeps the launch within one wave of two thread blocks
+  // per SM (at least 1, at most kMaxCluster, at most one tile per CTA).
+  int cs = static_cast<int>((2 * static_cast<int64_t>(device_sm_count())) / BH);
+  cs = max(1, min(cs, min(kMaxCluster, nt)));
+  while ((nt + cs - 1) / cs > kMaxScreenTiles && cs < kMaxCluster) ++cs;
   const int tpc = max(1, (nt + cs - 1) / cs);
   if (tpc > kMaxScreenTiles) return cudaErrorInvalidValue;
   const size_t smem = 128 + static_cast<size_t>(NST) * 2 * D * 32 * sizeof(float) + 2 * NST * sizeof(uint64_t) +
@@ -216,13 +244,6 @@ cudaError_t launch_tma_d(const ScreenCall& c, cudaStream_t st) {
 
 cudaError_t launch_screen_tma(const ScreenCall& c, cudaStream_t st) {
   const int64_t nb_cap = c.shape.capacity / c.shape.block_size;
-  // Staging pays off while the launch is latency bound: fewer thread blocks
-  // than about two per SM. Larger launches keep enough plain loads in flight
-  // (several blocks per SM), while the ring's shared memory allows one.
-  const int nb = static_cast<int>((c.n + c.shape.block_size - 1) / c.shape.block_size);
-  const int nt = (max(0, nb - c.n_local) + 31) / 32;
-  const int64_t ctas = static_cast<int64_t>(c.shape.batch) * c.shape.n_kv_heads * max(1, min(kMaxCluster, nt));
-  if (ctas >= 2 * static_cast<int64_t>(device_sm_count())) return cudaErrorNotSupported;
   // TMA wants 16-byte aligned rows and a 16-byte aligned base
   if (nb_cap % 4 != 0 || (reinterpret_cast<uintptr_t>(c.meta.mu) & 15) != 0 ||
       (reinterpret_cast<uintptr_t>(c.meta.var) & 15) != 0)
