@@ -3,8 +3,8 @@
 
 A step is the whole hot path for one batch of decode queries: threshold
 predictor (Eq. 1) -> block screening against the cached metadata (Eq. 5) ->
-block-sparse flash decoding with the sigmoid logit gate (Eq. 2-3) -> split
-combine. Default workload: GQA decode, batch 8, 32 query / 8 KV heads,
+block-sparse flash decoding with the sigmoid logit gate (Eq. 2-3), whose
+split partials are merged inside the same kernel. Default workload: GQA decode, batch 8, 32 query / 8 KV heads,
 d=128, 128K cached tokens, bf16 KV, block 32, predictor thresholds at ~38%
 head density (the 128K-context configuration).
 
@@ -38,7 +38,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20      # > 2x the 126 MB L2
-LAUNCHES_PER_STEP = {"predictor": 4, "const": 3}
+LAUNCHES_PER_STEP = {"predictor": 2, "const": 2}
 
 
 def parse_args():
@@ -341,26 +341,26 @@ def run_eta(args):
         return tau, stride, bias
 
     def step_phases(tau, stride, bias, ev):
-        """predict (if any) -> screen -> decode+combine, events between phases."""
+        """screen (forming the Eq. 1 thresholds itself when there is a
+        predictor) -> decode (split merge fused), events between phases."""
         ev[0].record(stream)
         if bias is not None:
-            binding.predict_tau(dec.shape, dw.q, dw.W, bias, dec.tau)
+            binding.screen_predict(dec.shape, dec.params, dw.q, dec.meta, w.n, dw.W, bias, dec.tau, dec.ws)
             t, s = dec.tau, w.Hq
         else:
+            binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, tau, stride, dec.ws)
             t, s = tau, stride
         ev[1].record(stream)
-        binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, t, s, dec.ws)
-        ev[2].record(stream)
         binding.decode_screened(dec.shape, dec.params, dw.q, dw.K, dw.V, w.n, t, s, dec.out, dec.ws)
-        ev[3].record(stream)
+        ev[2].record(stream)
 
     def time_sparse(density, sample_clocks=False):
         tau, stride, bias = thresholds(density)
         for _ in range(args.warmup):
             flush.zero_()
-            step_phases(tau, stride, bias, [torch.cuda.Event(enable_timing=True) for _ in range(4)])
+            step_phases(tau, stride, bias, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
         torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
         clk = ClockSampler(local) if sample_clocks else None
         barrier(world)
         torch.cuda.synchronize()
@@ -372,26 +372,24 @@ def run_eta(args):
         torch.cuda.synchronize()
         barrier(world)
         clocks = clk.stop() if clk else None
-        tot = sum(e[0].elapsed_time(e[3]) for e in evs) / args.steps
-        pre = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-        scr = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-        dec_t = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+        tot = sum(e[0].elapsed_time(e[2]) for e in evs) / args.steps
+        scr = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        dec_t = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
         # counts for the byte model (untimed extra screen with count outputs)
         ucnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=dev)
         hcnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=dev)
         if bias is not None:
-            binding.predict_tau(dec.shape, dw.q, dw.W, bias, dec.tau)
-            t, s = dec.tau, w.Hq
+            binding.screen_predict(dec.shape, dec.params, dw.q, dec.meta, w.n, dw.W, bias, dec.tau, dec.ws,
+                                   union_cnt=ucnt, active_cnt=hcnt)
         else:
-            t, s = tau, stride
-        binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, t, s, dec.ws, union_cnt=ucnt,
-                       active_cnt=hcnt)
+            binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, tau, stride, dec.ws, union_cnt=ucnt,
+                           active_cnt=hcnt)
         torch.cuda.synchronize()
         bm = byte_model(w, ucnt.cpu().numpy(), hcnt.cpu().numpy(), S)
         st = dec.device_status()
         if st != 0:
             raise RuntimeError(f"device status {st} after timed steps")
-        return {"ms": tot, "ms_predict": pre, "ms_screen": scr, "ms_decode": dec_t, "bytes": bm,
+        return {"ms": tot, "ms_screen": scr, "ms_decode": dec_t, "bytes": bm,
                 "clocks": clocks, "tau": (tau, stride, bias)}
 
     def time_dense():
@@ -457,9 +455,10 @@ def run_eta(args):
                    "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
         "effective_hbm_gbs": bm["step_read"] / (ms * 1e-3) / 1e9,
         "d_head": bm["d_head"], "d_union": bm["d_union"], "union_blocks": bm["union_blocks"],
-        "phases_ms": {"predict": main["ms_predict"], "screen": main["ms_screen"],
-                      "decode_combine": main["ms_decode"]},
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel (+combine, timed together)",
+        "phases_ms": {("screen+predict" if w.tau_mode == "predictor" else "screen"): main["ms_screen"],
+                      "decode": main["ms_decode"]},
+        "roofline": {"bound": "hbm",
+                     "kernel": ("decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel") + " (split merge fused)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind, "traffic": measured_traffic(w.name, bm["union_blocks"]),
                      "bytes_per_launch": bm["decode_kernel"]},

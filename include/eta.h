@@ -158,8 +158,12 @@ ETA_API eta_status_t eta_predict_tau(const eta_shape_t* shape, const void* q, co
  * resolved on the current device). Returns 0 for an invalid shape. */
 ETA_API size_t eta_decode_workspace_bytes(const eta_shape_t* shape, const eta_params_t* params);
 
-/* Clear the workspace's device status word (stream-ordered). Call once after
- * allocating a workspace; eta_read_device_status clears it as well. */
+/* Zero the workspace header (stream-ordered): the device status word and the
+ * per-(batch, kv head) counters of split partials that the decode kernel
+ * leaves at zero after every complete call. Call once after allocating a
+ * workspace. After a call whose device status was not ETA_OK,
+ * eta_read_device_status clears the header again. ws_bytes below the header
+ * size (33,024 bytes) gives ETA_ERR_WORKSPACE. */
 ETA_API eta_status_t eta_workspace_init(void* workspace, size_t ws_bytes, eta_stream_t stream);
 
 /*
@@ -185,8 +189,8 @@ ETA_API eta_status_t eta_screen(const eta_shape_t* shape, const eta_params_t* pa
 /*
  * eta_decode_sparse — one decode step of ETA (Figure 1 right, Figure 6):
  * screen (as eta_screen), then a flash-decoding pass over the admitted blocks
- * only, then a combine of the split partials. For query head h over the
- * tokens s < n of its admitted blocks (Eq. 2-3):
+ * only, whose split partials are merged in the same kernel. For query head h
+ * over the tokens s < n of its admitted blocks (Eq. 2-3):
  *   S_s = <q, k_s> / sqrt(d)
  *   g_s = S_s if s = t, else S_s * sigmoid(beta * (S_s - tau))
  *   out = sum_s exp(g_s - max g) v_s / sum_s exp(g_s - max g)       (fp32)
@@ -200,7 +204,36 @@ ETA_API eta_status_t eta_decode_sparse(const eta_shape_t* shape, const eta_param
                                        eta_stream_t stream);
 
 /*
- * eta_decode_screened — the decode and combine half of eta_decode_sparse:
+ * eta_screen_predict — eta_predict_tau and eta_screen in one launch
+ * (Methodology §1 Eq. 1, then §4 Eq. 5): every screening thread block forms
+ * the thresholds of its own query-head group from q, W and bias, with exactly
+ * eta_predict_tau's arithmetic and order, and screens against tau - a.
+ *   W, bias : as eta_predict_tau
+ *   tau_out : [B][Hq] fp32 out, the thresholds (bit-identical to
+ *             eta_predict_tau's); pass it to eta_decode_screened with a
+ *             batch stride of Hq
+ * Other arguments, outputs and errors as eta_screen.
+ */
+ETA_API eta_status_t eta_screen_predict(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                        eta_meta_t meta, int64_t n_tokens, const float* W, const float* bias,
+                                        float* tau_out, const eta_screen_out_t* out, void* workspace,
+                                        size_t ws_bytes, eta_stream_t stream);
+
+/*
+ * eta_decode_sparse_predict — one decode step with learned thresholds
+ * (Eq. 1-5): eta_screen_predict, then the decode of eta_decode_sparse gated
+ * by the thresholds it formed. Two launches; the result equals
+ * eta_predict_tau followed by eta_decode_sparse with tau_batch_stride = Hq.
+ *   tau_out : [B][Hq] fp32 out, the thresholds
+ */
+ETA_API eta_status_t eta_decode_sparse_predict(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                               const void* k, const void* v, eta_meta_t meta, int64_t n_tokens,
+                                               const float* W, const float* bias, float* tau_out, float* out,
+                                               const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
+                                               eta_stream_t stream);
+
+/*
+ * eta_decode_screened — the decode half of eta_decode_sparse:
  * attend over the union lists that the last eta_screen call wrote into this
  * workspace. That call must have used the same shape, params, q, n_tokens
  * and tau (the gate reads tau here); with them, eta_screen followed by
@@ -237,7 +270,8 @@ ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params
  * the array: calls whose kernels overlap on the GPU (unordered streams) race
  * and must not be issued. The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress); make it before any stream capture.
- * Each call clears the scratch status word first. device_status (nullable,
+ * Each call clears the scratch header (status word and partial counters)
+ * first. device_status (nullable,
  * device memory) receives this call's device status word, stream-ordered.
  * Other arguments and results as eta_decode_sparse.
  */
@@ -249,7 +283,8 @@ ETA_API eta_status_t eta_decode_sparse_static(const eta_shape_t* shape, const et
                                               eta_stream_t stream);
 
 /* Synchronise `stream`, read the workspace's device status word into *status
- * (host pointer) and clear it. Returns ETA_ERR_CUDA if the copy fails. */
+ * (host pointer) and clear it (the whole header when it was not ETA_OK).
+ * Returns ETA_ERR_CUDA if the copy fails. */
 ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t stream, eta_status_t* status);
 
 #ifdef __cplusplus

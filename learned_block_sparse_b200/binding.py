@@ -70,6 +70,11 @@ def _load():
     L.eta_decode_sparse.restype = st
     L.eta_decode_sparse.argtypes = [P(Shape), P(Params), vp, vp, vp, Meta, i64, vp, i64, vp, P(ScreenOut),
                                     vp, sz, vp]
+    L.eta_screen_predict.restype = st
+    L.eta_screen_predict.argtypes = [P(Shape), P(Params), vp, Meta, i64, vp, vp, vp, P(ScreenOut), vp, sz, vp]
+    L.eta_decode_sparse_predict.restype = st
+    L.eta_decode_sparse_predict.argtypes = [P(Shape), P(Params), vp, vp, vp, Meta, i64, vp, vp, vp, vp,
+                                            P(ScreenOut), vp, sz, vp]
     L.eta_decode_screened.restype = st
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
@@ -85,7 +90,8 @@ def _load():
 lib = _load()
 EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta_predict_tau",
             "eta_decode_workspace_bytes", "eta_workspace_init", "eta_screen", "eta_decode_sparse",
-            "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static")
+            "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static",
+            "eta_screen_predict", "eta_decode_sparse_predict")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -169,6 +175,25 @@ def screen(shape: Shape, params: Params, q, meta, n_tokens: int, tau: torch.Tens
                           _ptr(ws), ws.numel(), _stream(stream)), "eta_screen")
 
 
+def screen_predict(shape: Shape, params: Params, q, meta, n_tokens: int, W: torch.Tensor, bias: torch.Tensor,
+                   tau_out: torch.Tensor, ws: torch.Tensor, stream=None, **outs) -> None:
+    so = _screen_out(**outs)
+    _check(lib.eta_screen_predict(ctypes.byref(shape), ctypes.byref(params), _ptr(q),
+                                  Meta(*(m.data_ptr() for m in meta)), n_tokens, _ptr(W), _ptr(bias), _ptr(tau_out),
+                                  ctypes.byref(so) if so is not None else None, _ptr(ws), ws.numel(),
+                                  _stream(stream)), "eta_screen_predict")
+
+
+def decode_sparse_predict(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, W: torch.Tensor,
+                          bias: torch.Tensor, tau_out: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+                          stream=None, **outs) -> None:
+    so = _screen_out(**outs)
+    _check(lib.eta_decode_sparse_predict(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                         Meta(*(m.data_ptr() for m in meta)), n_tokens, _ptr(W), _ptr(bias),
+                                         _ptr(tau_out), _ptr(out), ctypes.byref(so) if so is not None else None,
+                                         _ptr(ws), ws.numel(), _stream(stream)), "eta_decode_sparse_predict")
+
+
 def decode_sparse(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, tau: torch.Tensor,
                   tau_batch_stride: int, out: torch.Tensor, ws: torch.Tensor, stream=None, **outs) -> None:
     so = _screen_out(**outs)
@@ -213,7 +238,7 @@ def read_device_status(ws: torch.Tensor, stream=None) -> int:
 class EtaDecoder:
     """One attention layer's decode state: the KV cache geometry, its block
     metadata and a workspace. ``step`` runs one decode step (predictor or given
-    thresholds -> screen -> block-sparse decode -> combine) through the C ABI."""
+    thresholds -> screen -> block-sparse decode) through the C ABI."""
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity,
                  kv_dtype=torch.bfloat16, q_dtype=torch.bfloat16, beta=5.0, z=1.0, offset_a=0.0,
@@ -244,12 +269,15 @@ class EtaDecoder:
     def step(self, q, k, v, n_tokens: int, tau: Optional[torch.Tensor] = None, W=None, bias=None,
              tau_batch_stride: Optional[int] = None, out: Optional[torch.Tensor] = None, **outs) -> torch.Tensor:
         """Sparse decode step. Thresholds: ``tau`` ([B][Hq], or [Hq] per-head
-        constants) or the predictor (``W``, ``bias``)."""
+        constants) or the predictor (``W``, ``bias``), formed inside the
+        screening launch and left in ``self.tau``."""
+        o = self.out if out is None else out
         if tau is None:
-            tau = self.predict_tau(q, W, bias)
+            decode_sparse_predict(self.shape, self.params, q, k, v, self.meta, n_tokens, W, bias, self.tau, o,
+                                  self.ws, **outs)
+            return o
         if tau_batch_stride is None:
             tau_batch_stride = 0 if tau.dim() == 1 else self.shape.n_q_heads
-        o = self.out if out is None else out
         decode_sparse(self.shape, self.params, q, k, v, self.meta, n_tokens, tau, tau_batch_stride, o, self.ws,
                       **outs)
         return o

@@ -56,11 +56,11 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int d, int64_t nb_cap, int S) {
   WsLayout L;
   const size_t BH = static_cast<size_t>(B) * Hkv, BHq = static_cast<size_t>(B) * Hq;
   size_t off = 0;
-  L.status = off;     off += round_up(sizeof(int32_t));
+  L.status = off;     off += 256;
+  L.seg_done = off;   off += round_up(kMaxBH * sizeof(int32_t));
   L.union_list = off; off += round_up(BH * static_cast<size_t>(nb_cap) * sizeof(uint32_t));
   L.union_cnt = off;  off += round_up(BH * sizeof(int32_t));
   L.head_cnt = off;   off += round_up(BHq * sizeof(int32_t));
-  L.prefix = off;     off += round_up((BH + 1) * sizeof(int32_t));
   L.o_part = off;     off += round_up(BHq * static_cast<size_t>(S) * d * sizeof(float));
   L.ml_part = off;    off += round_up(BHq * static_cast<size_t>(S) * sizeof(float2));
   L.total = off;
@@ -74,7 +74,7 @@ Workspace ws_carve(void* base, const WsLayout& L) {
   w.union_list = reinterpret_cast<uint32_t*>(p + L.union_list);
   w.union_cnt = reinterpret_cast<int32_t*>(p + L.union_cnt);
   w.head_cnt = reinterpret_cast<int32_t*>(p + L.head_cnt);
-  w.prefix = reinterpret_cast<int32_t*>(p + L.prefix);
+  w.seg_done = reinterpret_cast<int32_t*>(p + L.seg_done);
   w.o_part = reinterpret_cast<float*>(p + L.o_part);
   w.ml_part = reinterpret_cast<float2*>(p + L.ml_part);
   return w;
@@ -118,10 +118,11 @@ eta_status_t check_params(const eta_params_t* p) {
 }
 
 // Shapes the decode kernel can stage (two stages of a K and a V block plus its
-// fixed shared memory) and index (prefix table of B*Hkv entries).
+// fixed shared memory) and index (prefix table and partial counters of B*Hkv
+// entries).
 eta_status_t check_decode_shape(const eta_shape_t* s, bool dense) {
   const int BH = s->batch * s->n_kv_heads;
-  if (!dense && BH > kMaxBH) return ETA_ERR_UNSUPPORTED;
+  if (BH > kMaxBH) return ETA_ERR_UNSUPPORTED;
   const int G = s->n_q_heads / s->n_kv_heads;
   const size_t tile = static_cast<size_t>(s->block_size) * s->head_dim * elem_bytes(s->kv_dtype);
   const size_t fixed = static_cast<size_t>(8) * G * (s->head_dim + 2) * 4 + 16 +
@@ -174,7 +175,8 @@ eta_status_t check_meta(const eta_meta_t& m) {
 
 eta_status_t do_screen(const eta_shape_t* s, const eta_params_t* p, const void* q, eta_meta_t meta, int64_t n,
                        const float* tau, int64_t tau_stride, const eta_screen_out_t* out, const Workspace& w,
-                       cudaStream_t st) {
+                       cudaStream_t st, const float* W = nullptr, const float* bias = nullptr,
+                       float* tau_out = nullptr) {
   ScreenCall c;
   c.shape = *s;
   c.z = p->z;
@@ -185,6 +187,9 @@ eta_status_t do_screen(const eta_shape_t* s, const eta_params_t* p, const void* 
   c.n = n;
   c.tau = tau;
   c.tau_stride = tau_stride;
+  c.W = W;
+  c.bias = bias;
+  c.tau_out = tau_out;
   if (out != nullptr) c.out = *out;
   else std::memset(&c.out, 0, sizeof(c.out));
   c.ws = w;
@@ -198,6 +203,33 @@ eta_status_t check_common_decode(const eta_shape_t* s, const eta_params_t* p, co
   ETA_TRY(check_tokens(s, n));
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return ETA_ERR_INVALID_ARG;
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(q, elem_bytes(s->q_dtype)) || !aligned(out, 16))
+    return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+eta_status_t do_sparse_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k,
+                              const void* v, int64_t n, const float* tau, int64_t tau_stride, float* out,
+                              const Workspace& w, cudaStream_t st) {
+  DecodeCall c;
+  c.shape = *s;
+  c.beta = p->beta;
+  c.q = q;
+  c.k = k;
+  c.v = v;
+  c.n = n;
+  c.tau = tau;
+  c.tau_stride = tau_stride;
+  c.out = out;
+  c.ws = w;
+  c.S = resolve_splits(p);
+  c.dense = false;
+  return from_cuda(launch_decode(c, st));
+}
+
+eta_status_t check_predictor(const eta_shape_t* s, const void* q, const float* W, const float* bias,
+                             const float* tau) {
+  if (q == nullptr || W == nullptr || bias == nullptr || tau == nullptr) return ETA_ERR_INVALID_ARG;
+  if (!aligned(q, elem_bytes(s->q_dtype)) || !aligned(W, 4) || !aligned(bias, 4) || !aligned(tau, 4))
     return ETA_ERR_INVALID_ARG;
   return ETA_OK;
 }
@@ -234,13 +266,7 @@ ETA_API eta_status_t eta_build_block_meta(const eta_shape_t* shape, const void* 
 ETA_API eta_status_t eta_predict_tau(const eta_shape_t* shape, const void* q, const float* W, const float* bias,
                                      float* tau, eta_stream_t stream) {
   ETA_TRY(check_shape(shape));
-  if (q == nullptr || W == nullptr || bias == nullptr || tau == nullptr) return ETA_ERR_INVALID_ARG;
-  if (!aligned(q, elem_bytes(shape->q_dtype)) || !aligned(W, 4) || !aligned(bias, 4) || !aligned(tau, 4))
-    return ETA_ERR_INVALID_ARG;
-  // the kernel stages one batch row of queries (Hq*d fp32) in shared memory
-  if (static_cast<size_t>(shape->n_q_heads) * shape->head_dim * 4 + 8192 >
-      static_cast<size_t>(device_max_smem_optin()))
-    return ETA_ERR_UNSUPPORTED;
+  ETA_TRY(check_predictor(shape, q, W, bias, tau));
   return from_cuda(launch_predict(*shape, q, W, bias, tau, stream));
 }
 
@@ -252,8 +278,8 @@ ETA_API size_t eta_decode_workspace_bytes(const eta_shape_t* shape, const eta_pa
 }
 
 ETA_API eta_status_t eta_workspace_init(void* workspace, size_t ws_bytes, eta_stream_t stream) {
-  if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < 256) return ETA_ERR_WORKSPACE;
-  return from_cuda(cudaMemsetAsync(workspace, 0, sizeof(int32_t), stream));
+  if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < kWsHeaderBytes) return ETA_ERR_WORKSPACE;
+  return from_cuda(cudaMemsetAsync(workspace, 0, kWsHeaderBytes, stream));
 }
 
 ETA_API eta_status_t eta_screen(const eta_shape_t* shape, const eta_params_t* params, const void* q,
@@ -286,20 +312,40 @@ ETA_API eta_status_t eta_decode_sparse(const eta_shape_t* shape, const eta_param
   ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
   const Workspace w = ws_carve(workspace, L);
   ETA_TRY(do_screen(shape, params, q, meta, n_tokens, tau, tau_batch_stride, extra, w, stream));
-  DecodeCall c;
-  c.shape = *shape;
-  c.beta = params->beta;
-  c.q = q;
-  c.k = k;
-  c.v = v;
-  c.n = n_tokens;
-  c.tau = tau;
-  c.tau_stride = tau_batch_stride;
-  c.out = out;
-  c.ws = w;
-  c.S = resolve_splits(params);
-  c.dense = false;
-  return from_cuda(launch_decode(c, stream));
+  return do_sparse_decode(shape, params, q, k, v, n_tokens, tau, tau_batch_stride, out, w, stream);
+}
+
+ETA_API eta_status_t eta_screen_predict(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                        eta_meta_t meta, int64_t n_tokens, const float* W, const float* bias,
+                                        float* tau_out, const eta_screen_out_t* out, void* workspace,
+                                        size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_shape(shape));
+  ETA_TRY(check_params(params));
+  ETA_TRY(check_tokens(shape, n_tokens));
+  ETA_TRY(check_screen_shape(shape));
+  ETA_TRY(check_meta(meta));
+  ETA_TRY(check_predictor(shape, q, W, bias, tau_out));
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_screen(shape, params, q, meta, n_tokens, nullptr, 0, out, ws_carve(workspace, L), stream, W, bias,
+                   tau_out);
+}
+
+ETA_API eta_status_t eta_decode_sparse_predict(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                               const void* k, const void* v, eta_meta_t meta, int64_t n_tokens,
+                                               const float* W, const float* bias, float* tau_out, float* out,
+                                               const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
+                                               eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k, v, n_tokens, out));
+  ETA_TRY(check_screen_shape(shape));
+  ETA_TRY(check_decode_shape(shape, false));
+  ETA_TRY(check_meta(meta));
+  ETA_TRY(check_predictor(shape, q, W, bias, tau_out));
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  const Workspace w = ws_carve(workspace, L);
+  ETA_TRY(do_screen(shape, params, q, meta, n_tokens, nullptr, 0, extra, w, stream, W, bias, tau_out));
+  return do_sparse_decode(shape, params, q, k, v, n_tokens, tau_out, shape->n_q_heads, out, w, stream);
 }
 
 ETA_API eta_status_t eta_decode_screened(const eta_shape_t* shape, const eta_params_t* params, const void* q,
@@ -311,20 +357,8 @@ ETA_API eta_status_t eta_decode_screened(const eta_shape_t* shape, const eta_par
   if (tau == nullptr || tau_batch_stride < 0 || !aligned(tau, 4)) return ETA_ERR_INVALID_ARG;
   WsLayout L;
   ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
-  DecodeCall c;
-  c.shape = *shape;
-  c.beta = params->beta;
-  c.q = q;
-  c.k = k;
-  c.v = v;
-  c.n = n_tokens;
-  c.tau = tau;
-  c.tau_stride = tau_batch_stride;
-  c.out = out;
-  c.ws = ws_carve(workspace, L);
-  c.S = resolve_splits(params);
-  c.dense = false;
-  return from_cuda(launch_decode(c, stream));
+  return do_sparse_decode(shape, params, q, k, v, n_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L),
+                          stream);
 }
 
 ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params_t* params, const void* q,
@@ -358,7 +392,9 @@ ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t 
   cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return ETA_ERR_CUDA;
-  e = cudaMemsetAsync(const_cast<void*>(workspace), 0, sizeof(int32_t), stream);
+  // After a device error a call may have stopped between counting partials:
+  // clear the counters too.
+  e = cudaMemsetAsync(const_cast<void*>(workspace), 0, v == 0 ? sizeof(int32_t) : kWsHeaderBytes, stream);
   if (e != cudaSuccess) return ETA_ERR_CUDA;
   *status = static_cast<eta_status_t>(v);
   return ETA_OK;

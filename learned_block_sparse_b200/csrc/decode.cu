@@ -1,17 +1,18 @@
 // Block-sparse flash decoding over the admitted blocks (Figure 1 right,
-// Figure 6), with the ETA logit gate of Eq. 2-3 and an online softmax, then a
-// combine of the split partials.
+// Figure 6), with the ETA logit gate of Eq. 2-3 and an online softmax, and the
+// merge of the split partials in the same kernel.
 //
 // Work split. The admitted (union) blocks of all (batch, kv head) pairs form
 // one flat sequence of T entries; thread block k of S takes the contiguous
 // range [k*T/S, (k+1)*T/S), so every SM streams the same number of blocks
 // whatever the per-head densities are. Where a range crosses a (batch, kv head)
 // boundary the thread block emits one partial (running max, running sum,
-// unnormalised output) per query head; the combine kernel merges a head's
-// partials, which come from consecutive thread blocks.
+// unnormalised output) per query head; the thread block that writes the last
+// partial of a segment merges them (finish_segment), and a segment inside one
+// range is written out directly.
 //
 // This file holds the CUDA-core consumer (fp32 K/V, or bf16 K/V with fp32
-// queries), the combine kernel and the dispatch; bf16 K/V with bf16 queries
+// queries) and the dispatch; bf16 K/V with bf16 queries
 // go to the tensor-core consumer in decode_mma.cu.
 //
 // Pipeline. Warp 8 is the producer: one lane issues two 1-D TMA bulk copies
@@ -36,7 +37,6 @@ namespace {
 
 constexpr int kNW = 8;                       // consumer warps
 constexpr int kDecThreads = (kNW + 1) * 32;  // + one producer warp
-constexpr int kCombineWarps = 4;
 
 template <typename KV, int D, int G, bool DENSE>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs a) {
@@ -82,8 +82,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     return DENSE ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
   };
   const int64_t T = pre(BH);
-  if (!DENSE && blockIdx.x == 0)
-    for (int i = tid; i <= BH; i += kDecThreads) a.prefix_out[i] = s_pre[i];
   const int S = gridDim.x;
   const int kc = blockIdx.x;
   const int64_t lo = static_cast<int64_t>(kc) * T / S;
@@ -257,25 +255,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
         }
       }
       named_barrier_sync(1, kNW * 32);
-      const int b = cur / a.Hkv, kvh = cur % a.Hkv;
-      const int slotk = kc - range_of(pre(cur), T, S);
-      for (int idx = tid; idx < G * D; idx += kNW * 32) {
-        const int g = idx / D, e = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNW; ++w) M = fmaxf(M, s_mm[w * G + g]);
-        float o = 0.0f, L = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kNW; ++w) {
-          const float c = M == -INFINITY ? 0.0f : exp2f(s_mm[w * G + g] - M);
-          o = fmaf(c, s_macc[(w * G + g) * D + e], o);
-          L = fmaf(c, s_ml[w * G + g], L);
-        }
-        const int64_t row = (static_cast<int64_t>(b) * a.Hq + kvh * G + g) * S + slotk;
-        a.o_part[row * D + e] = o;
-        if (e == 0) a.ml_part[row] = make_float2(M, L);
-      }
-      named_barrier_sync(1, kNW * 32);
+      finish_segment<D, G, kNW>(a, cur, pre(cur), pre(cur + 1), lo, T, S, s_macc, s_mm, s_ml, s_abort + 1);
       if (p + 1 < hi) {
         do {
           ++cur;
@@ -285,60 +265,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
       }
     }
   }
-}
-
-struct CombineArgs {
-  const float* o_part;
-  const float2* ml_part;
-  const int32_t* prefix;
-  float* out;
-  int B, Hq, Hkv, nb, S;
-  int dense;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const CombineArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kCombineWarps + warp;
-  if (row >= a.B * a.Hq) return;
-  const int b = row / a.Hq, hq = row % a.Hq;
-  const int G = a.Hq / a.Hkv;
-  const int seg = b * a.Hkv + hq / G;
-  const int BH = a.B * a.Hkv;
-  const int64_t p0 = a.dense ? static_cast<int64_t>(seg) * a.nb : a.prefix[seg];
-  const int64_t p1 = a.dense ? static_cast<int64_t>(seg + 1) * a.nb : a.prefix[seg + 1];
-  const int64_t T = a.dense ? static_cast<int64_t>(BH) * a.nb : a.prefix[BH];
-  const int k0 = range_of(p0, T, a.S);
-  const int nsl = range_of(p1 - 1, T, a.S) - k0 + 1;
-  const float2* ml = a.ml_part + static_cast<int64_t>(row) * a.S;
-  // A range k is empty when floor(k*T/S) == floor((k+1)*T/S) (only when T < S):
-  // its thread block wrote no partial, so its slot is skipped.
-  auto empty_range = [&](int s) {
-    const int64_t k = k0 + s;
-    return (k * T) / a.S == ((k + 1) * T) / a.S;
-  };
-  float M = -INFINITY;
-  for (int s = lane; s < nsl; s += 32)
-    if (!empty_range(s)) M = fmaxf(M, ml[s].x);
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-  constexpr int PL = D / 32;
-  float o[PL];
-#pragma unroll
-  for (int e = 0; e < PL; ++e) o[e] = 0.0f;
-  float L = 0.0f;
-  const float* op = a.o_part + static_cast<int64_t>(row) * a.S * D;
-  for (int s = 0; s < nsl; ++s) {
-    if (empty_range(s)) continue;
-    const float2 v = ml[s];
-    const float c = (v.x == -INFINITY) ? 0.0f : exp2f(v.x - M);
-    L = fmaf(c, v.y, L);
-#pragma unroll
-    for (int e = 0; e < PL; ++e) o[e] = fmaf(c, op[static_cast<int64_t>(s) * D + lane * PL + e], o[e]);
-  }
-  const float inv = 1.0f / L;
-#pragma unroll
-  for (int e = 0; e < PL; ++e) a.out[static_cast<int64_t>(row) * D + lane * PL + e] = o[e] * inv;
 }
 
 template <typename KV, int D, int G, bool DENSE>
@@ -370,26 +296,6 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   return cudaSuccess;
 }
 
-cudaError_t launch_combine(const DecodeCall& c, cudaStream_t st) {
-  const eta_shape_t& s = c.shape;
-  CombineArgs ca;
-  ca.o_part = c.ws.o_part;
-  ca.ml_part = c.ws.ml_part;
-  ca.prefix = c.ws.prefix;
-  ca.out = c.out;
-  ca.B = s.batch;
-  ca.Hq = s.n_q_heads;
-  ca.Hkv = s.n_kv_heads;
-  ca.nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
-  ca.S = c.S;
-  ca.dense = c.dense ? 1 : 0;
-  const int rows = s.batch * s.n_q_heads;
-  const unsigned grid = static_cast<unsigned>((rows + kCombineWarps - 1) / kCombineWarps);
-  if (s.head_dim == 128) combine_kernel<128><<<grid, kCombineWarps * 32, 0, st>>>(ca);
-  else combine_kernel<64><<<grid, kCombineWarps * 32, 0, st>>>(ca);
-  return cudaGetLastError();
-}
-
 template <typename KV, int D, bool DENSE>
 cudaError_t launch_decode_g(const DecodeCall& c, cudaStream_t st) {
   switch (c.shape.n_q_heads / c.shape.n_kv_heads) {
@@ -409,15 +315,10 @@ cudaError_t launch_decode_kd(const DecodeCall& c, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st) {
-  cudaError_t e;
-  if (c.shape.kv_dtype == ETA_BF16 && c.shape.q_dtype == ETA_BF16)
-    e = launch_decode_mma(c, st);
-  else if (c.shape.kv_dtype == ETA_BF16)
-    e = c.dense ? launch_decode_kd<Bf16Raw, true>(c, st) : launch_decode_kd<Bf16Raw, false>(c, st);
-  else
-    e = c.dense ? launch_decode_kd<float, true>(c, st) : launch_decode_kd<float, false>(c, st);
-  if (e != cudaSuccess) return e;
-  return launch_combine(c, st);
+  if (c.shape.kv_dtype == ETA_BF16 && c.shape.q_dtype == ETA_BF16) return launch_decode_mma(c, st);
+  if (c.shape.kv_dtype == ETA_BF16)
+    return c.dense ? launch_decode_kd<Bf16Raw, true>(c, st) : launch_decode_kd<Bf16Raw, false>(c, st);
+  return c.dense ? launch_decode_kd<float, true>(c, st) : launch_decode_kd<float, false>(c, st);
 }
 
 }  // namespace eta

@@ -1,7 +1,8 @@
 // Pieces shared by the two decode kernels (CUDA-core consumer for fp32 K/V,
 // tensor-core consumer for bf16 K/V): arguments, the flat split of admitted
 // blocks over thread blocks, the on-chip prefix of the per-(batch, kv head)
-// counts, and the producer loop that walks this thread block's range.
+// counts, the producer loop that walks this thread block's range, and the
+// split-K merge that the thread block writing a segment's last partial runs.
 #pragma once
 
 #include <cmath>
@@ -20,7 +21,8 @@ struct DecodeArgs {
   const int32_t* union_cnt;
   float* o_part;
   float2* ml_part;
-  int32_t* prefix_out;
+  float* out;
+  int32_t* seg_done;
   int32_t* status;
   int64_t cap, n, tau_stride;
   int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
@@ -61,6 +63,98 @@ __device__ __forceinline__ void block_prefix(const int32_t* cnt, int32_t* s_pre,
       run += __shfl_sync(kFull, v, 31);
     }
     if (lane == 0) s_pre[0] = 0;
+  }
+}
+
+// The partials of a segment [p0, p1): one per thread block whose range meets
+// it, numbered from 0 in range order. With T >= S no range is empty and the
+// ranges k0 = range_of(p0) .. range_of(p1 - 1) each give one. With T < S a
+// range holds at most one position, so the partials are simply the segment's
+// positions: the thread block whose range starts at `lo` writes slot lo - p0.
+struct SegSpan {
+  int slot, parts;
+};
+__device__ __forceinline__ SegSpan seg_span(int64_t p0, int64_t p1, int64_t lo, int64_t T, int S) {
+  SegSpan r;
+  if (T >= S) {
+    const int k0 = range_of(p0, T, S);
+    r.slot = static_cast<int>(blockIdx.x) - k0;
+    r.parts = range_of(p1 - 1, T, S) - k0 + 1;
+  } else {
+    r.slot = static_cast<int>(lo - p0);
+    r.parts = static_cast<int>(p1 - p0);
+  }
+  return r;
+}
+
+// Epilogue of one segment (batch, kv head) in a thread block, called by its NW
+// consumer warps (named barrier 1) once each warp has left its running max
+// (log2 units), sum and unnormalised output rows in s_mm / s_ml / s_macc.
+// The warps' states are merged; a segment that lies inside this thread block's
+// range is normalised and written to `out` at once. Otherwise this range's
+// partial (m, l, o) goes to the workspace and is counted in seg_done[seg]; the
+// thread block that counts the segment's last partial merges all of them in
+// range order (a fixed order, so the result does not depend on which thread
+// block finishes last: flash-decoding's split-K reduction) and re-arms the
+// counter for the next call.
+template <int D, int G, int NW>
+__device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int64_t p0, int64_t p1, int64_t lo,
+                                               int64_t T, int S, const float* s_macc, const float* s_mm,
+                                               const float* s_ml, volatile int* s_flag) {
+  constexpr int kThr = NW * 32;
+  const int tid = threadIdx.x;
+  const int b = seg / a.Hkv, kvh = seg % a.Hkv;
+  const int64_t hq0 = static_cast<int64_t>(b) * a.Hq + kvh * G;
+  const SegSpan sp = seg_span(p0, p1, lo, T, S);
+  for (int idx = tid; idx < G * D; idx += kThr) {
+    const int g = idx / D, e = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_mm[w * G + g]);
+    float ov = 0.0f, L = 0.0f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      const float c = M == -INFINITY ? 0.0f : exp2f(s_mm[w * G + g] - M);
+      ov = fmaf(c, s_macc[(w * G + g) * D + e], ov);
+      L = fmaf(c, s_ml[w * G + g], L);
+    }
+    if (sp.parts == 1) {
+      a.out[(hq0 + g) * D + e] = ov * (1.0f / L);
+    } else {
+      const int64_t prow = (hq0 + g) * S + sp.slot;
+      a.o_part[prow * D + e] = ov;
+      if (e == 0) a.ml_part[prow] = make_float2(M, L);
+    }
+  }
+  if (sp.parts == 1) {
+    named_barrier_sync(1, kThr);  // s_macc is rewritten by the next segment
+    return;
+  }
+  __threadfence();  // this thread's partial is visible before the count
+  named_barrier_sync(1, kThr);
+  if (tid == 0) {
+    const int done = atomicAdd(a.seg_done + seg, 1) + 1;
+    const int last = done == sp.parts ? 1 : 0;
+    if (last) atomicExch(a.seg_done + seg, 0);
+    *s_flag = last;
+  }
+  named_barrier_sync(1, kThr);
+  if (*s_flag == 0) return;
+  __threadfence();
+  for (int idx = tid; idx < G * D; idx += kThr) {
+    const int g = idx / D, e = idx % D;
+    const float2* ml = a.ml_part + (hq0 + g) * S;
+    const float* op = a.o_part + (hq0 + g) * S * D + e;
+    float M = -INFINITY;
+    for (int s = 0; s < sp.parts; ++s) M = fmaxf(M, __ldcg(ml + s).x);
+    float o = 0.0f, L = 0.0f;
+    for (int s = 0; s < sp.parts; ++s) {
+      const float2 v = __ldcg(ml + s);
+      const float c = v.x == -INFINITY ? 0.0f : exp2f(v.x - M);
+      L = fmaf(c, v.y, L);
+      o = fmaf(c, __ldcg(op + static_cast<int64_t>(s) * D), o);
+    }
+    a.out[(hq0 + g) * D + e] = o * (1.0f / L);
   }
 }
 
@@ -148,7 +242,8 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.union_cnt = c.ws.union_cnt;
   a.o_part = c.ws.o_part;
   a.ml_part = c.ws.ml_part;
-  a.prefix_out = c.ws.prefix;
+  a.out = c.out;
+  a.seg_done = c.ws.seg_done;
   a.status = c.ws.status;
   a.cap = s.capacity;
   a.n = c.n;

@@ -148,8 +148,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
     return DENSE ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
   };
   const int64_t T = pre(BH);
-  if (!DENSE && blockIdx.x == 0)
-    for (int i = tid; i <= BH; i += kMmaThreads) a.prefix_out[i] = s_pre[i];
   const int S = gridDim.x;
   const int kc = blockIdx.x;
   const int64_t lo = static_cast<int64_t>(kc) * T / S;
@@ -221,25 +219,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
       }
     }
     named_barrier_sync(1, kMW * 32);
-    const int b = seg / a.Hkv, kvh = seg % a.Hkv;
-    const int slotk = kc - range_of(pre(seg), T, S);
-    for (int idx = tid; idx < G * D; idx += kMW * 32) {
-      const int g = idx / D, e = idx % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kMW; ++w) M = fmaxf(M, s_mm[w * G + g]);
-      float ov = 0.0f, L = 0.0f;
-#pragma unroll
-      for (int w = 0; w < kMW; ++w) {
-        const float c = M == -INFINITY ? 0.0f : exp2f(s_mm[w * G + g] - M);
-        ov = fmaf(c, s_macc[(w * G + g) * D + e], ov);
-        L = fmaf(c, s_ml[w * G + g], L);
-      }
-      const int64_t prow = (static_cast<int64_t>(b) * a.Hq + kvh * G + g) * S + slotk;
-      a.o_part[prow * D + e] = ov;
-      if (e == 0) a.ml_part[prow] = make_float2(M, L);
-    }
-    named_barrier_sync(1, kMW * 32);
+    finish_segment<D, G, kMW>(a, seg, pre(seg), pre(seg + 1), lo, T, S, s_macc, s_mm, s_ml, s_abort + 1);
   };
 
   // gate in log2 units: g = S * sigmoid(beta (S - tau)) * log2(e)

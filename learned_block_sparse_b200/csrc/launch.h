@@ -17,13 +17,13 @@ struct Workspace {
   uint32_t* union_list;   // [B*Hkv][nb_cap] (block << 8) | head mask
   int32_t* union_cnt;     // [B*Hkv]
   int32_t* head_cnt;      // [B*Hq]
-  int32_t* prefix;        // [B*Hkv + 1] exclusive prefix of union_cnt (decode -> combine)
+  int32_t* seg_done;      // [kMaxBH] partials counted per (batch, kv head); zero between calls
   float* o_part;          // [B*Hq][S][d] unnormalised partial outputs
   float2* ml_part;        // [B*Hq][S] (running max in log2 units, running sum)
 };
 
 struct WsLayout {
-  size_t status, union_list, union_cnt, head_cnt, prefix, o_part, ml_part, total;
+  size_t status, seg_done, union_list, union_cnt, head_cnt, o_part, ml_part, total;
 };
 
 WsLayout ws_layout(int B, int Hq, int Hkv, int d, int64_t nb_cap, int S);
@@ -60,6 +60,9 @@ struct ScreenCall {
   int64_t n;
   const float* tau;
   int64_t tau_stride;
+  const float* W;         // non-null: form tau by Eq. 1 inside the screen (tau ignored)
+  const float* bias;
+  float* tau_out;         // [B][Hq], written when W is non-null
   eta_screen_out_t out;   // optional outputs (fields may be null)
   Workspace ws;
 };
@@ -83,6 +86,9 @@ cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st);
 
 // Largest B*Hkv the decode kernel's on-chip prefix table holds.
 constexpr int kMaxBH = 8192;
+// The workspace starts with a fixed header, the part that must be zero before
+// a call: the status word (own 256-byte line) and the seg_done counters.
+constexpr size_t kWsHeaderBytes = 256 + kMaxBH * sizeof(int32_t);
 // Largest number of 32-block tiles one screening thread block holds.
 constexpr int kMaxScreenTiles = 1024;
 constexpr int kMaxCluster = 8;

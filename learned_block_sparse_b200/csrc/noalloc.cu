@@ -14,10 +14,10 @@
 // The scratch is one file-scope __device__ array of kStaticScratchBytes. Every
 // GPU that loads the library holds it until the process exits. All calls on a
 // device share it and it keeps the last call's contents: each call clears the
-// status word (the only part that must start at zero; everything else is
-// written before it is read within a call). Calls whose kernels overlap on
-// the GPU (different streams, no ordering between them) race on the array and
-// must not be issued.
+// workspace header (status word and partial counters, the only parts that must
+// start at zero; everything else is written before it is read within a call).
+// Calls whose kernels overlap on the GPU (different streams, no ordering
+// between them) race on the array and must not be issued.
 //
 // Host code cannot use the array's name as a device address: the first call on
 // each device looks the address up with cudaGetSymbolAddress (with that device
@@ -70,7 +70,7 @@ extern "C" ETA_API eta_status_t eta_decode_sparse_static(const eta_shape_t* shap
   if (need > kStaticScratchBytes) return ETA_ERR_WORKSPACE;  // shape too large for the fixed scratch
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return ETA_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, sizeof(int32_t), stream) != cudaSuccess) return ETA_ERR_CUDA;
+  if (eta_workspace_init(ws, kStaticScratchBytes, stream) != ETA_OK) return ETA_ERR_CUDA;
   const eta_status_t st = eta_decode_sparse(shape, params, q, k, v, meta, n_tokens, tau, tau_batch_stride, out, extra,
                                             ws, kStaticScratchBytes, stream);
   if (st != ETA_OK) return st;

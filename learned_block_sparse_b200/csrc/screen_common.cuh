@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "launch.h"
+#include "tau_chain.cuh"
 
 namespace eta {
 
@@ -21,6 +22,9 @@ struct ScreenArgs {
   const float* maxn;
   const float* tau;
   int64_t tau_stride;
+  const float* W;      // non-null: thresholds by Eq. 1 in the prologue
+  const float* bias;
+  float* tau_out;
   float z, s, offset_a;
   int Hq, Hkv, nb, ns, nb_cap, tiles_per_cta;
   uint32_t* ws_union;
@@ -48,6 +52,8 @@ struct ScreenSmem {
   float* taut;   // [G] tau - a
   int* tot;      // [G+1] this CTA's admitted counts
   int* base;     // [G+1] counts of lower-ranked CTAs
+  float* tau;    // [G] Eq. 1 thresholds (when formed in the prologue)
+  float* part;   // [32][G+1] Eq. 1 partials
   int* tcnt;     // [tpc][G+1] per-tile counts -> offsets
   uint8_t* mask; // [tpc*32] head mask of every block
   __device__ ScreenSmem(unsigned char* p, int tpc) {
@@ -55,19 +61,25 @@ struct ScreenSmem {
     qq = q + G * D;
     qn = qq + G * D;
     taut = qn + 16;
-    tot = reinterpret_cast<int*>(taut + 16);
+    tau = taut + 16;
+    part = tau + 16;
+    tot = reinterpret_cast<int*>(part + 32 * (G + 1));
     base = tot + 16;
     tcnt = base + 16;
     mask = reinterpret_cast<uint8_t*>(tcnt + tpc * (G + 1));
   }
-  static constexpr size_t fixed_bytes() { return (2 * G * D + 32) * sizeof(float) + 32 * sizeof(int); }
+  static constexpr size_t fixed_bytes() {
+    return (2 * G * D + 48 + 32 * (G + 1)) * sizeof(float) + 32 * sizeof(int);
+  }
   static size_t bytes(int tpc) {
     return fixed_bytes() + static_cast<size_t>(tpc) * (G + 1) * sizeof(int) + static_cast<size_t>(tpc) * 32;
   }
 };
 
 // Stage the group's queries, their squares, norms and thresholds. All threads.
-template <int D, int G>
+// With a.W set, the group's thresholds are formed here by Eq. 1 (chains with
+// kBatch loads in flight) and the cluster's first thread block writes them out.
+template <int D, int G, int kBatch>
 __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
                                                 int nthreads) {
   const int tid = threadIdx.x;
@@ -77,7 +89,21 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
     sm.q[i] = x;
     sm.qq[i] = __fmul_rn(x, x);
   }
-  __syncthreads();
+  if (a.W != nullptr) {
+    const int Hd = a.Hq * D;
+    const int64_t row = static_cast<int64_t>(b) * Hd;
+    if (a.q_dtype == ETA_BF16)
+      predict_heads<kBatch>(static_cast<const uint16_t*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part,
+                            sm.tau, nthreads);
+    else
+      predict_heads<kBatch>(static_cast<const float*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part,
+                            sm.tau, nthreads);
+    if (tid < G && cooperative_groups::this_cluster().block_rank() == 0)
+      a.tau_out[static_cast<int64_t>(b) * a.Hq + kvh * G + tid] = sm.tau[tid];
+  } else {
+    if (tid < G) sm.tau[tid] = a.tau[b * a.tau_stride + kvh * G + tid];
+    __syncthreads();
+  }
   if (tid < G) {
     float qn = 0.0f;  // sum of q_i^2 by fused multiply-adds in increasing i
     for (int e0 = 0; e0 < D; e0 += 16) {
@@ -88,7 +114,7 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
       for (int c = 0; c < 16; ++c) qn = __fmaf_rn(x[c], x[c], qn);
     }
     sm.qn[tid] = __fsqrt_rn(qn);
-    sm.taut[tid] = __fsub_rn(a.tau[b * a.tau_stride + kvh * G + tid], a.offset_a);
+    sm.taut[tid] = __fsub_rn(sm.tau[tid], a.offset_a);
   }
   __syncthreads();
 }
@@ -219,6 +245,9 @@ inline ScreenArgs make_screen_args(const ScreenCall& c, int nb, int ns, int tpc)
   a.maxn = c.meta.maxnorm;
   a.tau = c.tau;
   a.tau_stride = c.tau_stride;
+  a.W = c.W;
+  a.bias = c.bias;
+  a.tau_out = c.tau_out;
   a.z = c.z;
   a.s = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.head_dim)));
   a.offset_a = c.offset_a;

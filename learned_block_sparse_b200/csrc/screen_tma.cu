@@ -87,7 +87,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
   const int first = my_tiles < NST ? my_tiles : NST;
   if (warp == CW && lane == 0)
     for (int it = 0; it < first; ++it) issue_tile(it);
-  screen_prologue<D, G>(a, sm, b, kvh, NT);  // ends with __syncthreads
+  screen_prologue<D, G, 64>(a, sm, b, kvh, NT);  // ends with __syncthreads
 
   if (warp == CW) {
     // ------------------------------------------------------------ producer

@@ -203,8 +203,48 @@ def test_repeat_calls_identical():
     tau = torch.zeros((w.B, w.Hq), device="cuda")
     a = dw.step(tau=tau, stride=w.Hq).clone()
     b = dw.step(tau=tau, stride=w.Hq).clone()
+    d1 = dw.dense().clone()
+    d2 = dw.dense().clone()
     torch.cuda.synchronize()
-    assert torch.equal(a, b)
+    assert torch.equal(a, b) and torch.equal(d1, d2)
+    # the split-partial counters in the workspace header are back at zero
+    counters = dw.dec.ws[256:256 + 4 * 8192].view(torch.int32)
+    assert int(torch.count_nonzero(counters)) == 0
+
+
+@pytest.mark.parametrize("dtype,G,bs", [("bf16", 4, 32), ("bf16", 8, 64), ("f32", 2, 16), ("bf16", 1, 64)])
+def test_thresholds_in_screen_equal_separate_predictor(dtype, G, bs):
+    """eta_decode_sparse_predict (Eq. 1 formed inside the screening launch)
+    gives the thresholds, lists and outputs of eta_predict_tau followed by
+    eta_decode_sparse, bit for bit; both thresholds match the oracle's."""
+    w = synth.Workload("p", dtype, 3, 4 * G, 4, 64 if G == 8 else 128, bs * 90 + 7, bs, z=1.0,
+                       tau_mode="predictor", densities=(0.3,), seed=90 + G + bs, offset_std=synth.SQRT_HALF)
+    dw = DeviceWorkload(w, keep_host=True)
+    meta = parity.oracle_meta(w, dw.K_host)
+    tau, _, bias = parity.oracle_thresholds(w, dw.q_host, meta, 0.3, W=dw.W)
+    b_dev = torch.as_tensor(bias, device="cuda")
+    nb_cap = w.capacity // w.bs
+
+    def outs():
+        return dict(active_idx=torch.full((w.B, w.Hq, nb_cap), -1, dtype=torch.int32, device="cuda"),
+                    active_cnt=torch.zeros((w.B, w.Hq), dtype=torch.int32, device="cuda"),
+                    union_cnt=torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda"))
+
+    o1 = outs()
+    fused = dw.dec.step(dw.q, dw.K, dw.V, w.n, W=dw.W, bias=b_dev, **o1).clone()
+    tau_fused = dw.dec.tau.clone()
+    tau_sep = torch.empty_like(tau_fused)
+    binding.predict_tau(dw.dec.shape, dw.q, dw.W, b_dev, tau_sep)
+    o2 = outs()
+    sep = dw.dec.step(dw.q, dw.K, dw.V, w.n, tau=tau_sep, tau_batch_stride=w.Hq, **o2).clone()
+    torch.cuda.synchronize()
+    assert dw.dec.device_status() == 0
+    want = np.asarray(tau, np.float32).reshape(w.B, w.Hq).view(np.int32)
+    assert np.array_equal(tau_fused.cpu().numpy().view(np.int32), want)
+    assert np.array_equal(tau_sep.cpu().numpy().view(np.int32), want)
+    for k in o1:
+        assert torch.equal(o1[k], o2[k]), k
+    assert torch.equal(fused, sep)
 
 
 # ----------------------------------------------------------------- full size
