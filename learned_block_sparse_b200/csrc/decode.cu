@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
       bulk_g2s(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes, kb + off, bytes, &s_full[st], pol);
       bulk_g2s(s_tiles + (static_cast<size_t>(st) * 2 + 1) * tile_bytes, vb + off, bytes, &s_full[st], pol);
     };
-    producer_loop<G, DENSE>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
+    producer_loop<G, DENSE, 4>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
     return;
   }
 

@@ -159,19 +159,21 @@ __device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int
 }
 
 // Producer warp: walk positions [lo, hi) in order. Lanes 0..PL-1 each take
-// every PL-th position (position lo + i goes to lane i % PL, PL = 4, or less
-// when the ring has fewer stages, so PL consecutive positions never share a
-// stage and are armed in parallel): wait until the position's stage is free,
+// every PL-th position (position lo + i goes to lane i % PL; PL = kMaxPL, or
+// less when the ring has fewer stages, so PL consecutive positions never share
+// a stage and are armed in parallel): wait until the position's stage is free,
 // publish (block, head mask, rows, segment) in s_info and call
 // issue(stage, segment, block, rows), which must arm s_full[stage] (arrive +
 // expected bytes) and start the copies. The warp reads the union list 32
 // entries at a time, one batch ahead. A stage's r-th reuse waits for the
 // consumer release that completed the empty barrier's phase r-1.
-template <int G, bool DENSE, typename SegOf, typename Pre, typename Issue>
+template <int G, bool DENSE, int kMaxPL, typename SegOf, typename Pre, typename Issue>
 __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, int64_t hi, int NST,
                                               uint64_t* s_empty, int4* s_info, int* s_abort, SegOf seg_of,
                                               Pre pre, Issue issue, uint64_t* s_full) {
-  const int PL = NST >= 4 ? 4 : (NST >= 2 ? 2 : 1);  // issuing lanes
+  static_assert(kMaxPL == 1 || kMaxPL == 2 || kMaxPL == 4 || kMaxPL == 8, "issuing lanes divide 32");
+  int PL = kMaxPL;  // issuing lanes
+  while (PL > NST) PL >>= 1;
   const int lane = threadIdx.x & 31;
   auto load_entry = [&](int64_t p, int& seg, uint32_t& e) {
     seg = 0;

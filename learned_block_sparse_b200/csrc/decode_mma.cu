@@ -15,7 +15,7 @@
 // [b rows][64 dims], 128-byte swizzle) of each admitted block's K and V into a
 // ring of stages; with that swizzle the 8 rows an ldmatrix reads sit in 8
 // different bank groups. Consumer warps own whole blocks (position i of the
-// range goes to warp i mod 4): S = Q K^T from ldmatrix'd K fragments, scale,
+// range goes to warp i mod (number of consumer warps)): S = Q K^T from ldmatrix'd K fragments, scale,
 // gate, online softmax in log2 units on the accumulator fragments, then
 // O += P V with P split into bf16 high and low parts so the probabilities keep
 // ~16 bits of precision: the high part sits in tile rows 0-7 and the low part
@@ -34,8 +34,14 @@ namespace eta {
 
 namespace {
 
-constexpr int kMW = 4;                       // consumer warps
-constexpr int kMmaThreads = (kMW + 1) * 32;  // + one producer warp
+// Consumer warps: 4, or 8 for 16-token blocks (8 KiB of K+V at d=128), whose
+// per-block latency chain needs more blocks in flight per SM; plus one
+// producer warp.
+template <int CH>
+struct MmaWarps {
+  static constexpr int kMW = CH == 16 ? 8 : 4;
+  static constexpr int kThreads = (kMW + 1) * 32;
+};
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar,
                                             uint64_t policy) {
@@ -105,13 +111,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D, int G, bool DENSE, int CH>
-__global__ void __launch_bounds__(kMmaThreads, 1)
+__global__ void __launch_bounds__(MmaWarps<CH>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   constexpr int KST = D / 16;  // k-steps of QK^T
   constexpr int NDT = D / 8;   // n-tiles of PV
   static_assert(G >= 1 && G <= 8, "group size");
   static_assert(CH == 16 || CH == 32, "keys per chunk");
+  constexpr int kMW = MmaWarps<CH>::kMW;
+  constexpr int kMmaThreads = MmaWarps<CH>::kThreads;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1)
         tma_load_2d(vt + h * bs * 128, &tmv, h * 64, y, &s_full[st], pol);
       }
     };
-    producer_loop<G, DENSE>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
+    producer_loop<G, DENSE, kMW>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
     return;
   }
 
@@ -403,6 +411,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
   const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
+  constexpr int kMW = MmaWarps<CH>::kMW;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 +
                        (DENSE ? 0 : static_cast<size_t>(BH + 1) * sizeof(int32_t)) + 1024;
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
@@ -426,7 +435,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH>));
   if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(c, nst);
-  decode_mma_kernel<D, G, DENSE, CH><<<c.S, kMmaThreads, smem, st>>>(a, tmk, tmv);
+  decode_mma_kernel<D, G, DENSE, CH><<<c.S, MmaWarps<CH>::kThreads, smem, st>>>(a, tmk, tmv);
   return cudaGetLastError();
 }
 
