@@ -24,7 +24,8 @@ __global__ void __launch_bounds__(kPredThreads)
   const int Hd = Hq * D;
   const int h0 = blockIdx.y * kHeadsPerBlock;
   const int NH = min(kHeadsPerBlock, Hq - h0);
-  predict_heads<64>(q + b * Hd, W, bias, Hq, Hd, h0, NH, part, tau_s, kPredThreads);
+  predict_heads<64>(q + b * Hd, W, bias, Hq, Hd, h0, NH, part, tau_s, static_cast<int>(threadIdx.x),
+                    kPredThreads, [] { __syncthreads(); });
   if (threadIdx.x < NH) tau[b * Hq + h0 + threadIdx.x] = tau_s[threadIdx.x];
 }
 

@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
 
   extern __shared__ __align__(16) unsigned char smem[];
   const ScreenSmem<D, G> sm(smem, tpc);
-  screen_prologue<D, G, 32>(a, sm, b, kvh, kScreenWarps * 32);
+  screen_prologue<D, G, 32, true>(a, sm, b, kvh, kScreenWarps * 32);
 
   const int nt = (a.ns + 31) / 32;
   const int t0 = cr * tpc;

@@ -76,10 +76,32 @@ struct ScreenSmem {
   }
 };
 
-// Stage the group's queries, their squares, norms and thresholds. All threads.
-// With a.W set, the group's thresholds are formed here by Eq. 1 (chains with
-// kBatch loads in flight) and the cluster's first thread block writes them out.
-template <int D, int G, int kBatch>
+// Eq. 1 thresholds of the group's heads (a.W set) by the `nthreads` threads
+// with relative index `rel`, synchronised by `sync`: sm.tau, sm.taut = tau - a,
+// and the cluster's first thread block writes tau to a.tau_out.
+template <int D, int G, int kBatch, typename Sync>
+__device__ __forceinline__ void screen_predict_tau(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
+                                                   int rel, int nthreads, Sync sync) {
+  const int Hd = a.Hq * D;
+  const int64_t row = static_cast<int64_t>(b) * Hd;
+  if (a.q_dtype == ETA_BF16)
+    predict_heads<kBatch>(static_cast<const uint16_t*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part,
+                          sm.tau, rel, nthreads, sync);
+  else
+    predict_heads<kBatch>(static_cast<const float*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part, sm.tau,
+                          rel, nthreads, sync);
+  if (rel < G) {
+    sm.taut[rel] = __fsub_rn(sm.tau[rel], a.offset_a);
+    if (cooperative_groups::this_cluster().block_rank() == 0)
+      a.tau_out[static_cast<int64_t>(b) * a.Hq + kvh * G + rel] = sm.tau[rel];
+  }
+}
+
+// Stage the group's queries, their squares and norms, and the thresholds
+// tau - a: read from a.tau, or (a.W set and kTauHere) formed by Eq. 1 with all
+// threads; with a.W set and !kTauHere the caller forms them (screen_predict_tau)
+// before any decision. All threads; ends with __syncthreads.
+template <int D, int G, int kBatch, bool kTauHere>
 __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
                                                 int nthreads) {
   const int tid = threadIdx.x;
@@ -89,21 +111,12 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
     sm.q[i] = x;
     sm.qq[i] = __fmul_rn(x, x);
   }
-  if (a.W != nullptr) {
-    const int Hd = a.Hq * D;
-    const int64_t row = static_cast<int64_t>(b) * Hd;
-    if (a.q_dtype == ETA_BF16)
-      predict_heads<kBatch>(static_cast<const uint16_t*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part,
-                            sm.tau, nthreads);
-    else
-      predict_heads<kBatch>(static_cast<const float*>(a.q) + row, a.W, a.bias, a.Hq, Hd, kvh * G, G, sm.part,
-                            sm.tau, nthreads);
-    if (tid < G && cooperative_groups::this_cluster().block_rank() == 0)
-      a.tau_out[static_cast<int64_t>(b) * a.Hq + kvh * G + tid] = sm.tau[tid];
-  } else {
-    if (tid < G) sm.tau[tid] = a.tau[b * a.tau_stride + kvh * G + tid];
-    __syncthreads();
+  if (a.W == nullptr) {
+    if (tid < G) sm.taut[tid] = __fsub_rn(a.tau[b * a.tau_stride + kvh * G + tid], a.offset_a);
+  } else if (kTauHere) {
+    screen_predict_tau<D, G, kBatch>(a, sm, b, kvh, tid, nthreads, [] { __syncthreads(); });
   }
+  __syncthreads();
   if (tid < G) {
     float qn = 0.0f;  // sum of q_i^2 by fused multiply-adds in increasing i
     for (int e0 = 0; e0 < D; e0 += 16) {
@@ -114,7 +127,6 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
       for (int c = 0; c < 16; ++c) qn = __fmaf_rn(x[c], x[c], qn);
     }
     sm.qn[tid] = __fsqrt_rn(qn);
-    sm.taut[tid] = __fsub_rn(sm.tau[tid], a.offset_a);
   }
   __syncthreads();
 }

@@ -28,6 +28,16 @@ template <int D> struct TmaScreenCfg;
 // 96 KB of stages: two thread blocks per SM.
 template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 3; };
 template <> struct TmaScreenCfg<64> { static constexpr int kCW = 3, kNST = 6; };
+// Warps that form the Eq. 1 thresholds (when the call passes a predictor)
+// while the ring streams the first tiles: the consumers score tiles and
+// release their stages without waiting for them, and wait only before the
+// first admission decision.
+constexpr int kTauWarps = 4;
+
+// Bytes between the stages and ScreenSmem: full and empty barriers, the
+// threshold barrier (+ 8 bytes padding), the abort flag (+ 12 bytes padding).
+template <int NST>
+constexpr size_t kTmaBarBytes = (2 * NST + 2) * sizeof(uint64_t) + 4 * sizeof(int);
 
 __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -38,12 +48,12 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
+__global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2)
     screen_tma_kernel(const ScreenArgs a, int32_t* status, const __grid_constant__ CUtensorMap tmu,
                       const __grid_constant__ CUtensorMap tvar) {
   constexpr int CW = TmaScreenCfg<D>::kCW;
   constexpr int NST = TmaScreenCfg<D>::kNST;
-  constexpr int NT = (CW + 1) * 32;
+  constexpr int NT = (CW + 1 + kTauWarps) * 32;  // consumers, producer, threshold warps
   constexpr uint32_t kBox = D * 32 * sizeof(float);  // one array's tile
   static_assert(NST % CW == 0, "stages must return to the same consumer warp");
   cg::cluster_group cluster = cg::this_cluster();
@@ -59,8 +69,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
   float* s_stage = reinterpret_cast<float*>(smem);  // [NST][2][D][32]
   uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * kBox);
   uint64_t* s_empty = s_full + NST;
-  int* s_abort = reinterpret_cast<int*>(s_empty + NST);
-  const ScreenSmem<D, G> sm(reinterpret_cast<unsigned char*>(s_abort + 4), tpc);
+  uint64_t* s_tau = s_empty + NST;  // completes when the thresholds are in sm.taut
+  int* s_abort = reinterpret_cast<int*>(s_tau + 2);
+  // the query rows are read as float4: ScreenSmem must start 16-byte aligned
+  static_assert((static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>) % 16 == 0, "ScreenSmem alignment");
+  const ScreenSmem<D, G> sm(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>, tpc);
 
   const int nt = (a.ns + 31) / 32;
   const int t0 = cr * tpc;
@@ -73,6 +86,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
     }
+    mbar_init(s_tau, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -87,9 +101,19 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
   const int first = my_tiles < NST ? my_tiles : NST;
   if (warp == CW && lane == 0)
     for (int it = 0; it < first; ++it) issue_tile(it);
-  screen_prologue<D, G, 64>(a, sm, b, kvh, NT);  // ends with __syncthreads
+  screen_prologue<D, G, 32, false>(a, sm, b, kvh, NT);  // ends with __syncthreads
+  const bool tau_later = a.W != nullptr;
 
-  if (warp == CW) {
+  if (warp > CW) {
+    // ----------------------------------------------------- threshold warps
+    if (tau_later) {
+      constexpr int kTauThreads = kTauWarps * 32;
+      screen_predict_tau<D, G, 32>(a, sm, b, kvh, tid - (CW + 1) * 32, kTauThreads,
+                                   [] { named_barrier_sync(2, kTauThreads); });
+      named_barrier_sync(2, kTauThreads);  // every taut written before the release
+      if (tid == (CW + 1) * 32) mbar_arrive(s_tau);
+    }
+  } else if (warp == CW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       int issued = first;
@@ -113,6 +137,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
     }
   } else {
     // ----------------------------------------------------------- consumers
+    bool tau_ok = !tau_later;
+    bool tau_waited = !tau_later;
     for (int it = warp; it < my_tiles; it += CW) {
       const int st = it % NST;
       const int blk = (t0 + it) * 32 + lane;
@@ -151,7 +177,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1) * 32, 2)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[st]);
-      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, blk, valid, dg, vg, M));
+      if (!tau_waited) {
+        tau_ok = mbar_wait_bounded(s_tau, 0u, s_abort, status);
+        tau_waited = true;
+      }
+      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, blk, valid && tau_ok, dg, vg, M));
     }
   }
   __syncthreads();
@@ -200,8 +230,8 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   while ((nt + cs - 1) / cs > kMaxScreenTiles && cs < kMaxCluster) ++cs;
   const int tpc = max(1, (nt + cs - 1) / cs);
   if (tpc > kMaxScreenTiles) return cudaErrorInvalidValue;
-  const size_t smem = 128 + static_cast<size_t>(NST) * 2 * D * 32 * sizeof(float) + 2 * NST * sizeof(uint64_t) +
-                      4 * sizeof(int) + ScreenSmem<D, G>::bytes(tpc);
+  const size_t smem = 128 + static_cast<size_t>(NST) * 2 * D * 32 * sizeof(float) + kTmaBarBytes<NST> +
+                      ScreenSmem<D, G>::bytes(tpc);
   if (smem > static_cast<size_t>(device_max_smem_optin())) return cudaErrorNotSupported;
   CUtensorMap tmu, tvar;
   const int64_t rows = static_cast<int64_t>(BH) * D;
@@ -214,7 +244,7 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(BH * cs));
-  cfg.blockDim = dim3((CW + 1) * 32);
+  cfg.blockDim = dim3((CW + 1 + kTauWarps) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

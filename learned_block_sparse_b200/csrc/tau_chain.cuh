@@ -50,28 +50,30 @@ __device__ __forceinline__ float tau_partial(const QT* __restrict__ qrow, const 
   return p;
 }
 
-// tau of heads h0 .. h0+NH-1 (NH <= 32) of one batch row into tau_s[0..NH).
-// Every thread of the block calls it (nthreads a multiple of 32, the call ends
-// with __syncthreads); part is shared scratch of 32*(NH+1) floats.
-template <int kBatch, typename QT>
+// tau of heads h0 .. h0+NH-1 (NH <= 32) of one batch row into tau_s[0..NH),
+// by the `nthreads` threads (a multiple of 32) whose index relative to the
+// first of them is `rel`; `sync()` must synchronise exactly those threads (it
+// is called twice, the second time before returning). part is shared scratch
+// of 32*(NH+1) floats.
+template <int kBatch, typename QT, typename Sync>
 __device__ __forceinline__ void predict_heads(const QT* __restrict__ qrow, const float* __restrict__ W,
                                               const float* __restrict__ bias, int Hq, int Hd, int h0, int NH,
-                                              float* part, float* tau_s, int nthreads) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+                                              float* part, float* tau_s, int rel, int nthreads, Sync sync) {
+  const int warp = rel >> 5, lane = rel & 31;
   // chain (l, g) = thread l*NH + g: neighbouring threads read neighbouring
   // heads of one row of W
-  for (int c = tid; c < 32 * NH; c += nthreads) {
+  for (int c = rel; c < 32 * NH; c += nthreads) {
     const int l = c / NH, g = c % NH;
     part[l * (NH + 1) + g] = tau_partial<kBatch>(qrow, W, Hq, Hd, l, h0 + g);
   }
-  __syncthreads();
+  sync();
   for (int g = warp; g < NH; g += nthreads >> 5) {
     float v = part[lane * (NH + 1) + g];
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(kFull, v, o));
     if (lane == 0) tau_s[g] = __fadd_rn(v, __ldg(bias + h0 + g));
   }
-  __syncthreads();
+  sync();
 }
 
 }  // namespace eta
