@@ -55,6 +55,9 @@ def parse_args():
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sweep", action="store_true", help="skip the other densities of the configuration")
+    p.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
+                   help="between steps: write 512 MiB, or write then read 512 MiB so the timed step "
+                        "does not also pay for writing back the flush's dirty lines")
     p.add_argument("--cpu-groups", type=int, default=64, help="(b, kv head) groups in the CPU sample")
     return p.parse_args()
 
@@ -333,7 +336,19 @@ def run_eta(args):
     dw = DeviceWorkload(w, device=dev, n_splits=args.n_splits)
     dec = dw.dec
     stream = torch.cuda.current_stream()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clean_buf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    class _Flush:
+        @staticmethod
+        def zero_():
+            # write > 2x L2 (evicts every line of the inputs), then read another
+            # buffer > L2 so the dirty lines of that write are written back
+            # before the timed region instead of inside it
+            flush_buf.zero_()
+            if args.l2_flush == "write+read":
+                clean_buf.sum()
+    flush = _Flush()
     S = args.n_splits or torch.cuda.get_device_properties(dev).multi_processor_count
 
     def thresholds(density):
@@ -452,7 +467,8 @@ def run_eta(args):
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller; see DESIGN.md input recipe)",
         "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
                    "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
-                   "l2": "flushed (512 MiB write) before every timed step", "parallelism": f"replicas x{world}"},
+                   "l2": ("flushed before every timed step: 512 MiB write" +
+                          (", then a 512 MiB read (no dirty lines left)" if args.l2_flush == "write+read" else "")), "parallelism": f"replicas x{world}"},
         "effective_hbm_gbs": bm["step_read"] / (ms * 1e-3) / 1e9,
         "d_head": bm["d_head"], "d_union": bm["d_union"], "union_blocks": bm["union_blocks"],
         "phases_ms": {("screen+predict" if w.tau_mode == "predictor" else "screen"): main["ms_screen"],
