@@ -49,7 +49,8 @@ def parse_args():
     p.add_argument("--impl", default="eta", choices=["eta", "reference"])
     p.add_argument("--config", type=int, default=3)
     p.add_argument("--batch", type=int, default=None, help="override the batch (config 5 sweep)")
-    p.add_argument("--density", type=float, default=0.38)
+    p.add_argument("--density", type=float, default=None,
+                   help="target admitted fraction (default: the middle density of the workload)")
     p.add_argument("--n-splits", type=int, default=0)
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-dense", action="store_true")
@@ -59,7 +60,12 @@ def parse_args():
                    help="between steps: write 512 MiB, or write then read 512 MiB so the timed step "
                         "does not also pay for writing back the flush's dirty lines")
     p.add_argument("--cpu-groups", type=int, default=64, help="(b, kv head) groups in the CPU sample")
-    return p.parse_args()
+    args = p.parse_args()
+    if args.density is None:
+        from learned_block_sparse_b200 import synth
+        ds = synth.WORKLOADS[args.config].densities
+        args.density = ds[len(ds) // 2]
+    return args
 
 
 # ----------------------------------------------------------------- plumbing
@@ -199,15 +205,21 @@ def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
     lists_read = 4 * blocks
     q = w.B * w.Hq * w.d * eb
     T = blocks
-    # partials: one per (query head, range it touches)
+    # split merge: a segment inside one range writes its output rows directly;
+    # one crossing ranges writes one (m, l, o) partial per range and head (read
+    # back once by the merging thread block, from L2)
     pre = np.concatenate([[0], np.cumsum(union_cnt.reshape(-1))])
-    slots = 0
+    partial_rows = 0
     for i in range(bh):
-        k0 = ((pre[i] + 1) * S - 1) // T
-        k1 = ((pre[i + 1]) * S - 1) // T
-        slots += sum(1 for k in range(int(k0), int(k1) + 1) if (k * T) // S != ((k + 1) * T) // S)
-    partials = slots * w.G * (w.d + 2) * 4
-    decode = kv + lists_read + q + partials
+        if T >= S:
+            parts = ((pre[i + 1]) * S - 1) // T - ((pre[i] + 1) * S - 1) // T + 1
+        else:
+            parts = pre[i + 1] - pre[i]
+        if parts > 1:
+            partial_rows += int(parts)
+    partials = partial_rows * w.G * (w.d + 2) * 4
+    out = w.B * w.Hq * w.d * 4
+    decode = kv + lists_read + q + partials + out
     meta = bh * w.n_screened * (2 * w.d + 1) * 4
     W = (w.Hq * w.d * w.Hq * 4 + w.Hq * 4) if w.tau_mode == "predictor" else 0
     step_read = kv + meta + lists_read + q * 2 + W

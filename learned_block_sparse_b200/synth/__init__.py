@@ -86,7 +86,7 @@ class Workload:
     bs: int              # block size b
     z: float             # screening confidence
     tau_mode: str        # "const" (per-head constant) or "predictor"
-    densities: tuple     # target fractions of screened blocks admitted per head
+    densities: tuple     # target fractions of screened blocks admitted (see density_kind)
     seed: int
     beta: float = 5.0
     n_local: int = 1
@@ -94,6 +94,7 @@ class Workload:
     n_needles: int = 0
     needle_scale: float = 3.0
     cap: Optional[int] = None    # allocated tokens per (b, kv head); default n rounded up to 4 blocks
+    density_kind: str = "head"   # "head": per query head; "union": of the GQA group's union
 
     @property
     def capacity(self) -> int:
@@ -128,7 +129,10 @@ class Workload:
 
 SQRT_HALF = math.sqrt(0.5)
 
-# The five decode configurations (names state the shapes).
+# The decode configurations (names state the shapes). 1-5 are the parity and
+# benchmark workloads; 6 is the attention shape of the pages' block-size /
+# chunk-size table (Table 10: batch 64, 512K tokens, 32 query / 4 KV heads of
+# dimension 64, blocks of 64), calibrated to the union densities quoted there.
 WORKLOADS = {
     1: Workload("tiny-f32-mha2-d64-n1024-b16", "f32", 1, 2, 2, 64, 1024, 16, z=1.5,
                 tau_mode="const", densities=(0.40,), seed=1001),
@@ -142,6 +146,9 @@ WORKLOADS = {
     5: Workload("mha16-d128-n64k-b16-const-sweep", "bf16", 1, 16, 16, 128, 65536, 16, z=1.5,
                 tau_mode="const", densities=(0.10, 0.25, 0.38, 0.60, 1.0), seed=1005,
                 offset_std=SQRT_HALF),
+    6: Workload("gqa32x4-d64-n512k-b64-B64", "bf16", 64, 32, 4, 64, 524288, 64, z=1.0,
+                tau_mode="predictor", densities=(0.16, 0.355, 0.512), seed=1006,
+                offset_std=SQRT_HALF, density_kind="union"),
 }
 WORKLOAD5_BATCHES = (1, 4, 16, 64)
 

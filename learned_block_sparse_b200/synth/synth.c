@@ -54,16 +54,24 @@ static inline double u53(uint32_t lo, uint32_t hi) {
   return ((double)(x >> 11) + 0.5) * (1.0 / 9007199254740992.0); /* in (0,1) */
 }
 
-/* standard normal number f of stream `stream` under `seed` */
-static inline double normal_at(uint64_t seed, uint32_t stream, uint64_t f) {
-  uint64_t pair = f >> 1;
+/* standard normal numbers 2*pair (cosine branch) and 2*pair + 1 (sine branch)
+ * of stream `stream` under `seed`: one Philox block, Box-Muller in double */
+static inline void normal_pair(uint64_t seed, uint32_t stream, uint64_t pair, double* z0, double* z1) {
   uint32_t w[4];
   philox4x32_10((uint32_t)pair, (uint32_t)(pair >> 32), stream, 0u,
                 (uint32_t)seed, (uint32_t)(seed >> 32), w);
   double u1 = u53(w[0], w[1]), u2 = u53(w[2], w[3]);
   double r = sqrt(-2.0 * log(u1));
   double th = 6.283185307179586476925286766559 * u2;
-  return (f & 1) ? r * sin(th) : r * cos(th);
+  *z0 = r * cos(th);
+  *z1 = r * sin(th);
+}
+
+/* standard normal number f of stream `stream` under `seed` */
+static inline double normal_at(uint64_t seed, uint32_t stream, uint64_t f) {
+  double z0, z1;
+  normal_pair(seed, stream, f >> 1, &z0, &z1);
+  return (f & 1) ? z1 : z0;
 }
 
 double synth_normal_at(uint64_t seed, uint32_t stream, uint64_t f) {
@@ -158,8 +166,8 @@ static void kv_range(void* p, int64_t lo, int64_t hi) {
   kv_ctx* c = (kv_ctx*)p;
   const int64_t d = c->d;
   const int G = (int)(c->Hq / c->H);
-  double qhat[1024];
-  int64_t cur_bh = -1;
+  double qhat[1024], off[1024], pair_hi = 0.0;
+  int64_t cur_bh = -1, cur_off = -1;
   for (int64_t lrow = lo; lrow < hi; ++lrow) {    /* lrow = ((b-b0)*H + h)*n + s */
     const int64_t row = lrow + c->b0 * c->H * c->n;
     int64_t bh = row / c->n, s = row % c->n;
@@ -182,9 +190,21 @@ static void kv_range(void* p, int64_t lo, int64_t hi) {
     const uint64_t f0 = (uint64_t)row * (uint64_t)d;
     const uint64_t foff = ((uint64_t)bh * (uint64_t)((c->n + c->bs - 1) / c->bs) + (uint64_t)blk) * (uint64_t)d;
     const int64_t o = ((bh - c->b0 * c->H) * c->cap + s) * d;
+    if (c->offset_std > 0.0 && (int64_t)foff != cur_off) {
+      /* the block's offset vector, drawn once per block */
+      for (int64_t i = 0; i < d; ++i) off[i] = normal_at(c->seed, c->off_stream, foff + (uint64_t)i);
+      cur_off = (int64_t)foff;
+    }
     for (int64_t i = 0; i < d; ++i) {
-      double x = normal_at(c->seed, c->stream, f0 + (uint64_t)i);
-      if (c->offset_std > 0.0) x += c->offset_std * normal_at(c->seed, c->off_stream, foff + (uint64_t)i);
+      double x;
+      if ((d & 1) == 0 && (i & 1) == 0) {   /* both numbers of a pair from one draw */
+        normal_pair(c->seed, c->stream, (f0 + (uint64_t)i) >> 1, &x, &pair_hi);
+      } else if ((d & 1) == 0) {
+        x = pair_hi;
+      } else {
+        x = normal_at(c->seed, c->stream, f0 + (uint64_t)i);
+      }
+      if (c->offset_std > 0.0) x += c->offset_std * off[i];
       if (is_needle) x += c->needle_scale * qhat[i];
       store(c->dst, c->dtype, o + i, x);
     }

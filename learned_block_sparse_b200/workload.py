@@ -65,30 +65,63 @@ class DeviceWorkload:
         return scores[:, :, :w.n_screened]
 
     @staticmethod
-    def _kth_largest(s: torch.Tensor, density: float) -> torch.Tensor:
+    def _kth_of_sorted(s: torch.Tensor, density: float) -> torch.Tensor:
+        """Per row of descending-sorted scores: the round(density*m)-th largest
+        (at least the first); -inf for density >= 1."""
         m = s.shape[-1]
         if density >= 1.0 or m == 0:
             return torch.full(s.shape[:-1], float("-inf"), dtype=torch.float32, device=s.device)
         k = max(1, int(round(density * m)))
-        return s.topk(k, dim=-1).values[..., -1]
+        return s[..., k - 1].contiguous()
+
+    def _union_density(self, sc: torch.Tensor, thr: torch.Tensor) -> float:
+        """Fraction of screened blocks in the GQA union when head h admits the
+        blocks with score >= thr[b][h]."""
+        w = self.w
+        adm = sc >= thr[:, :, None]
+        return adm.view(w.B, w.Hkv, w.G, -1).any(dim=2).float().mean().item()
 
     def calibrate(self, density: float):
-        """Thresholds admitting about `density` of each head's screened blocks,
-        pooled over the batch. Per-head constants: (tau [Hq], stride 0).
-        Predictor: returns (None, None, bias) with the bias shifted so that
-        score >= q.W + bias holds for that fraction; the caller runs the predictor."""
+        """Thresholds admitting about `density` of the screened blocks: of each
+        head's blocks pooled over the batch, or (density_kind "union") of the
+        GQA unions, by bisection on a common per-head density.
+        Per-head constants: (tau [Hq], stride 0). Predictor: returns
+        (None, None, bias) with the bias shifted so that score >= q.W + bias
+        holds for that fraction; the caller runs the predictor."""
         w = self.w
         sc = self.block_scores()
         if w.tau_mode == "const":
-            tau = self._kth_largest(sc.transpose(0, 1).reshape(w.Hq, -1), density).contiguous()
-            return tau, 0, None
-        tau0 = torch.empty((w.B, w.Hq), dtype=torch.float32, device=self.device)
-        binding.predict_tau(self.dec.shape, self.q, self.W, self.bias0, tau0)
-        # bias_h: the threshold, relative to each row's predicted tau, that admits
-        # the target fraction of the head's screened blocks pooled over the batch
-        shifted = (sc - tau0[:, :, None]).transpose(0, 1).reshape(w.Hq, -1)
-        bias = self._kth_largest(shifted, density).contiguous()
-        return None, None, bias
+            pooled = sc.transpose(0, 1).reshape(w.Hq, -1).sort(dim=-1, descending=True).values
+
+            def thr_of(rho):
+                return self._kth_of_sorted(pooled, rho)
+
+            def full(t):
+                return t[None, :].expand(w.B, w.Hq)
+        else:
+            tau0 = torch.empty((w.B, w.Hq), dtype=torch.float32, device=self.device)
+            binding.predict_tau(self.dec.shape, self.q, self.W, self.bias0, tau0)
+            # bias_h: the threshold, relative to each row's predicted tau, that admits
+            # the target fraction of the head's screened blocks pooled over the batch
+            shifted = (sc - tau0[:, :, None]).transpose(0, 1).reshape(w.Hq, -1).sort(dim=-1, descending=True).values
+
+            def thr_of(rho):
+                return self._kth_of_sorted(shifted, rho)
+
+            def full(bias):
+                return tau0 + bias[None, :]   # the predictor's fl(partial sum + bias)
+        rho = density
+        if w.density_kind == "union" and 0.0 < density < 1.0:
+            lo, hi = 0.0, density             # a head's density never exceeds its union's
+            for _ in range(24):
+                mid = 0.5 * (lo + hi)
+                if self._union_density(sc, full(thr_of(mid))) < density:
+                    lo = mid
+                else:
+                    hi = mid
+            rho = hi
+        t = thr_of(rho)
+        return (t, 0, None) if w.tau_mode == "const" else (None, None, t)
 
     # ------------------------------------------------------------- one step
     def step(self, tau=None, stride=None, bias=None, out=None, **outs) -> torch.Tensor:

@@ -100,11 +100,13 @@ def _reduced(i):
         3: base.replace(B=2, Hq=8, Hkv=2, n=32 * 150 + 5),
         4: base.replace(Hq=4, Hkv=4, n=64 * 100 + 63),
         5: base.replace(B=3, Hq=4, Hkv=4, n=16 * 300 + 9),
+        6: base.replace(B=2, n=64 * 120 + 9),
     }[i]
 
 
 @pytest.mark.parametrize("cfg,density", [(1, 0.40), (2, 0.38), (3, 0.20), (3, 0.38), (3, 0.60), (4, 0.38),
-                                         (5, 0.10), (5, 0.25), (5, 0.38), (5, 0.60), (5, 1.0)])
+                                         (5, 0.10), (5, 0.25), (5, 0.38), (5, 0.60), (5, 1.0), (6, 0.05),
+                                         (6, 0.2)])
 def test_workload_parity_reduced(cfg, density):
     r = _full_check(_reduced(cfg), density, dense=(cfg in (1, 4)))
     assert r["err"] <= parity.TOL[_reduced(cfg).dtype]
