@@ -34,12 +34,13 @@ namespace eta {
 
 namespace {
 
-// Consumer warps: 4, or 8 for 16-token blocks (8 KiB of K+V at d=128), whose
-// per-block latency chain needs more blocks in flight per SM; plus one
-// producer warp.
-template <int CH>
+// Consumer warps: 4, or 8 where a block carries more consumer work per byte
+// than a 32-token block at d=128: 16-token blocks (half the bytes per block
+// for the same fixed cost) and d=64 (twice the keys, hence twice the gate and
+// softmax work, per byte); plus one producer warp.
+template <int D, int CH>
 struct MmaWarps {
-  static constexpr int kMW = CH == 16 ? 8 : 4;
+  static constexpr int kMW = (CH == 16 || D == 64) ? 8 : 4;
   static constexpr int kThreads = (kMW + 1) * 32;
 };
 
@@ -111,15 +112,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 template <int D, int G, bool DENSE, int CH>
-__global__ void __launch_bounds__(MmaWarps<CH>::kThreads, 1)
+__global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   constexpr int KST = D / 16;  // k-steps of QK^T
   constexpr int NDT = D / 8;   // n-tiles of PV
   static_assert(G >= 1 && G <= 8, "group size");
   static_assert(CH == 16 || CH == 32, "keys per chunk");
-  constexpr int kMW = MmaWarps<CH>::kMW;
-  constexpr int kMmaThreads = MmaWarps<CH>::kThreads;
+  constexpr int kMW = MmaWarps<D, CH>::kMW;
+  constexpr int kMmaThreads = MmaWarps<D, CH>::kThreads;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -411,7 +412,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
   const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
-  constexpr int kMW = MmaWarps<CH>::kMW;
+  constexpr int kMW = MmaWarps<D, CH>::kMW;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 +
                        (DENSE ? 0 : static_cast<size_t>(BH + 1) * sizeof(int32_t)) + 1024;
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
@@ -435,7 +436,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH>));
   if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(c, nst);
-  decode_mma_kernel<D, G, DENSE, CH><<<c.S, MmaWarps<CH>::kThreads, smem, st>>>(a, tmk, tmv);
+  decode_mma_kernel<D, G, DENSE, CH><<<c.S, MmaWarps<D, CH>::kThreads, smem, st>>>(a, tmk, tmv);
   return cudaGetLastError();
 }
 
