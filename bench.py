@@ -377,7 +377,8 @@ def run_eta(args):
         else:
             binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, tau, stride, dec.ws)
             t, s = tau, stride
-        ev[1].record(stream)
+        if ev[1] is not None:   # an event between the launches also stops the decode starting early
+            ev[1].record(stream)
         binding.decode_screened(dec.shape, dec.params, dw.q, dw.K, dw.V, w.n, t, s, dec.out, dec.ws)
         ev[2].record(stream)
 
@@ -387,7 +388,9 @@ def run_eta(args):
             flush.zero_()
             step_phases(tau, stride, bias, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
         torch.cuda.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        # whole steps (the two launches back to back): the headline time
+        evs = [[torch.cuda.Event(enable_timing=True), None, torch.cuda.Event(enable_timing=True)]
+               for _ in range(args.steps)]
         clk = ClockSampler(local) if sample_clocks else None
         barrier(world)
         torch.cuda.synchronize()
@@ -400,8 +403,14 @@ def run_eta(args):
         barrier(world)
         clocks = clk.stop() if clk else None
         tot = sum(e[0].elapsed_time(e[2]) for e in evs) / args.steps
-        scr = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-        dec_t = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+        # the same steps with an event between the launches, for the phase split
+        pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            step_phases(tau, stride, bias, pevs[i])
+        torch.cuda.synchronize()
+        scr = sum(e[0].elapsed_time(e[1]) for e in pevs) / args.steps
+        dec_t = sum(e[1].elapsed_time(e[2]) for e in pevs) / args.steps
         # counts for the byte model (untimed extra screen with count outputs)
         ucnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=dev)
         hcnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=dev)

@@ -121,6 +121,18 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Programmatic dependent launch. The screening and decode kernels are launched
+// with cudaLaunchAttributeProgrammaticStreamSerialization, so each may start
+// (launch, shared-memory and barrier set-up) while the kernel before it on the
+// stream is still running. grid_dependency_wait() blocks until that kernel has
+// completed and its writes are visible (immediately when there is none): call
+// it before the first global read. allow_dependent_launch() lets the next
+// kernel on the stream begin launching.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   int* s_abort = reinterpret_cast<int*>(s_ml + kNW * G);
   int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
 
+  grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();
   if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kDecThreads);
   if (tid == 0) {
     *s_abort = 0;
@@ -289,11 +291,7 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   if (e != cudaSuccess) return e;
 
   const DecodeArgs a = make_decode_args(c, nst);
-  decode_kernel<KV, D, G, DENSE><<<c.S, kDecThreads, smem, st>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-
-  return cudaSuccess;
+  return launch_pdl(decode_kernel<KV, D, G, DENSE>, static_cast<unsigned>(c.S), kDecThreads, smem, st, a);
 }
 
 template <typename KV, int D, bool DENSE>

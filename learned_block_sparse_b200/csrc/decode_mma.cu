@@ -139,6 +139,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   int* s_abort = reinterpret_cast<int*>(s_ml + kMW * G);
   int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
 
+  grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();
   if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kMmaThreads);
   if (tid == 0) {
     *s_abort = 0;
@@ -436,8 +438,8 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH>));
   if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(c, nst);
-  decode_mma_kernel<D, G, DENSE, CH><<<c.S, MmaWarps<D, CH>::kThreads, smem, st>>>(a, tmk, tmv);
-  return cudaGetLastError();
+  return launch_pdl(decode_mma_kernel<D, G, DENSE, CH>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads, smem,
+                    st, a, tmk, tmv);
 }
 
 template <int D, bool DENSE, int CH>

@@ -45,6 +45,32 @@ inline cudaError_t allow_max_smem(std::atomic<uint64_t>& done, const void* fn) {
   return e;
 }
 
+// Launch attribute that lets a kernel start while the previous kernel on the
+// stream finishes (programmatic dependent launch). Only for kernels that call
+// grid_dependency_wait() before their first global read.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a = {};
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+// Launch `kernel` on `grid` x `block` threads with programmatic dependent launch.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 cudaError_t launch_build_meta(const eta_shape_t& s, const void* k, int64_t b0, int64_t b1, const eta_meta_t& m,
                               cudaStream_t st);
 

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
 
   extern __shared__ __align__(16) unsigned char smem[];
   const ScreenSmem<D, G> sm(smem, tpc);
+  grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();
   screen_prologue<D, G, 32, true>(a, sm, b, kvh, kScreenWarps * 32);
 
   const int nt = (a.ns + 31) / 32;

@@ -89,6 +89,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
     mbar_init(s_tau, 1);
     fence_mbar_init();
   }
+  grid_dependency_wait();  // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();
   __syncthreads();
   auto issue_tile = [&](int it) {
     const int st = it % NST;
@@ -247,13 +249,14 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   cfg.blockDim = dim3((CW + 1 + kTauWarps) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, screen_tma_kernel<D, G>, a, c.ws.status, tmu, tvar);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
