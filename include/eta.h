@@ -256,6 +256,45 @@ ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params
                                       eta_stream_t stream);
 
 /*
+ * Per-row lengths. The four calls below are eta_screen / eta_decode_sparse /
+ * eta_decode_screened / eta_decode_dense for a batch whose rows hold
+ * different numbers of cached tokens (the paged or continuous-batching case):
+ *   seq_lens   : [B] int32, device memory: tokens of row b including its
+ *                current token (t_b = seq_lens[b] - 1). Rows attend, screen
+ *                and are gated exactly as a call with n_tokens = seq_lens[b].
+ *                Read on the device, so a CUDA graph can replay the call
+ *                while the lengths change.
+ *   max_tokens : host upper bound of seq_lens, 1 <= max_tokens <= capacity;
+ *                sizes the launches. A length outside [1, max_tokens] sets
+ *                ETA_ERR_INVALID_ARG in the device status word and is clamped
+ *                to that range.
+ * Thresholds (eta_screen_ragged, eta_decode_sparse_ragged): with W == NULL
+ * they are tau / tau_batch_stride as in eta_screen; with W set they are
+ * formed by Eq. 1 as in eta_screen_predict (tau ignored, tau_out [B][Hq]
+ * written). Other arguments, outputs and errors as the uniform-length calls.
+ */
+ETA_API eta_status_t eta_screen_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                       eta_meta_t meta, const int32_t* seq_lens, int64_t max_tokens,
+                                       const float* tau, int64_t tau_batch_stride, const float* W,
+                                       const float* bias, float* tau_out, const eta_screen_out_t* out,
+                                       void* workspace, size_t ws_bytes, eta_stream_t stream);
+ETA_API eta_status_t eta_decode_sparse_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                              const void* k, const void* v, eta_meta_t meta,
+                                              const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                              int64_t tau_batch_stride, const float* W, const float* bias,
+                                              float* tau_out, float* out, const eta_screen_out_t* extra,
+                                              void* workspace, size_t ws_bytes, eta_stream_t stream);
+ETA_API eta_status_t eta_decode_screened_ragged(const eta_shape_t* shape, const eta_params_t* params,
+                                                const void* q, const void* k, const void* v,
+                                                const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                                int64_t tau_batch_stride, float* out, void* workspace,
+                                                size_t ws_bytes, eta_stream_t stream);
+ETA_API eta_status_t eta_decode_dense_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             int64_t max_tokens, const float* tau, int64_t tau_batch_stride,
+                                             float* out, void* workspace, size_t ws_bytes, eta_stream_t stream);
+
+/*
  * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and
  * without any device allocation. The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory when they

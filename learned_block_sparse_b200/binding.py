@@ -75,6 +75,16 @@ def _load():
     L.eta_decode_sparse_predict.restype = st
     L.eta_decode_sparse_predict.argtypes = [P(Shape), P(Params), vp, vp, vp, Meta, i64, vp, vp, vp, vp,
                                             P(ScreenOut), vp, sz, vp]
+    L.eta_screen_ragged.restype = st
+    L.eta_screen_ragged.argtypes = [P(Shape), P(Params), vp, Meta, vp, i64, vp, i64, vp, vp, vp, P(ScreenOut),
+                                    vp, sz, vp]
+    L.eta_decode_sparse_ragged.restype = st
+    L.eta_decode_sparse_ragged.argtypes = [P(Shape), P(Params), vp, vp, vp, Meta, vp, i64, vp, i64, vp, vp, vp,
+                                           vp, P(ScreenOut), vp, sz, vp]
+    L.eta_decode_screened_ragged.restype = st
+    L.eta_decode_screened_ragged.argtypes = [P(Shape), P(Params), vp, vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
+    L.eta_decode_dense_ragged.restype = st
+    L.eta_decode_dense_ragged.argtypes = [P(Shape), P(Params), vp, vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_screened.restype = st
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
@@ -91,7 +101,8 @@ lib = _load()
 EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta_predict_tau",
             "eta_decode_workspace_bytes", "eta_workspace_init", "eta_screen", "eta_decode_sparse",
             "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static",
-            "eta_screen_predict", "eta_decode_sparse_predict")
+            "eta_screen_predict", "eta_decode_sparse_predict", "eta_screen_ragged", "eta_decode_sparse_ragged",
+            "eta_decode_screened_ragged", "eta_decode_dense_ragged")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -194,6 +205,52 @@ def decode_sparse_predict(shape: Shape, params: Params, q, k, v, meta, n_tokens:
                                          _ptr(ws), ws.numel(), _stream(stream)), "eta_decode_sparse_predict")
 
 
+def _thr(tau, W, bias, tau_out):
+    """(tau, W, bias, tau_out) pointers of a per-row-length call."""
+    if W is not None:
+        return None, _ptr(W), _ptr(bias), _ptr(tau_out)
+    return _ptr(tau), None, None, None
+
+
+def screen_ragged(shape: Shape, params: Params, q, meta, seq_lens: torch.Tensor, max_tokens: int, ws: torch.Tensor,
+                  tau: Optional[torch.Tensor] = None, tau_batch_stride: int = 0, W=None, bias=None, tau_out=None,
+                  stream=None, **outs) -> None:
+    so = _screen_out(**outs)
+    t, w_, b_, to = _thr(tau, W, bias, tau_out)
+    _check(lib.eta_screen_ragged(ctypes.byref(shape), ctypes.byref(params), _ptr(q),
+                                 Meta(*(m.data_ptr() for m in meta)), _ptr(seq_lens), max_tokens, t,
+                                 tau_batch_stride, w_, b_, to, ctypes.byref(so) if so is not None else None,
+                                 _ptr(ws), ws.numel(), _stream(stream)), "eta_screen_ragged")
+
+
+def decode_sparse_ragged(shape: Shape, params: Params, q, k, v, meta, seq_lens: torch.Tensor, max_tokens: int,
+                         out: torch.Tensor, ws: torch.Tensor, tau: Optional[torch.Tensor] = None,
+                         tau_batch_stride: int = 0, W=None, bias=None, tau_out=None, stream=None, **outs) -> None:
+    so = _screen_out(**outs)
+    t, w_, b_, to = _thr(tau, W, bias, tau_out)
+    _check(lib.eta_decode_sparse_ragged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                        Meta(*(m.data_ptr() for m in meta)), _ptr(seq_lens), max_tokens, t,
+                                        tau_batch_stride, w_, b_, to, _ptr(out),
+                                        ctypes.byref(so) if so is not None else None, _ptr(ws), ws.numel(),
+                                        _stream(stream)), "eta_decode_sparse_ragged")
+
+
+def decode_screened_ragged(shape: Shape, params: Params, q, k, v, seq_lens: torch.Tensor, max_tokens: int,
+                           tau: torch.Tensor, tau_batch_stride: int, out: torch.Tensor, ws: torch.Tensor,
+                           stream=None) -> None:
+    _check(lib.eta_decode_screened_ragged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                          _ptr(seq_lens), max_tokens, _ptr(tau), tau_batch_stride, _ptr(out),
+                                          _ptr(ws), ws.numel(), _stream(stream)), "eta_decode_screened_ragged")
+
+
+def decode_dense_ragged(shape: Shape, params: Params, q, k, v, seq_lens: torch.Tensor, max_tokens: int,
+                        tau: Optional[torch.Tensor], tau_batch_stride: int, out: torch.Tensor, ws: torch.Tensor,
+                        stream=None) -> None:
+    _check(lib.eta_decode_dense_ragged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(seq_lens), max_tokens, _ptr(tau), tau_batch_stride, _ptr(out),
+                                       _ptr(ws), ws.numel(), _stream(stream)), "eta_decode_dense_ragged")
+
+
 def decode_sparse(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, tau: torch.Tensor,
                   tau_batch_stride: int, out: torch.Tensor, ws: torch.Tensor, stream=None, **outs) -> None:
     so = _screen_out(**outs)
@@ -267,27 +324,43 @@ class EtaDecoder:
         return self.tau
 
     def step(self, q, k, v, n_tokens: int, tau: Optional[torch.Tensor] = None, W=None, bias=None,
-             tau_batch_stride: Optional[int] = None, out: Optional[torch.Tensor] = None, **outs) -> torch.Tensor:
+             tau_batch_stride: Optional[int] = None, out: Optional[torch.Tensor] = None,
+             seq_lens: Optional[torch.Tensor] = None, **outs) -> torch.Tensor:
         """Sparse decode step. Thresholds: ``tau`` ([B][Hq], or [Hq] per-head
         constants) or the predictor (``W``, ``bias``), formed inside the
-        screening launch and left in ``self.tau``."""
+        screening launch and left in ``self.tau``. With ``seq_lens`` (int32
+        [B] on the device) row b holds seq_lens[b] tokens and ``n_tokens`` is
+        their upper bound."""
         o = self.out if out is None else out
+        if tau is not None and tau_batch_stride is None:
+            tau_batch_stride = 0 if tau.dim() == 1 else self.shape.n_q_heads
+        if seq_lens is not None:
+            if tau is None:
+                decode_sparse_ragged(self.shape, self.params, q, k, v, self.meta, seq_lens, n_tokens, o, self.ws,
+                                     W=W, bias=bias, tau_out=self.tau, **outs)
+            else:
+                decode_sparse_ragged(self.shape, self.params, q, k, v, self.meta, seq_lens, n_tokens, o, self.ws,
+                                     tau=tau, tau_batch_stride=tau_batch_stride, **outs)
+            return o
         if tau is None:
             decode_sparse_predict(self.shape, self.params, q, k, v, self.meta, n_tokens, W, bias, self.tau, o,
                                   self.ws, **outs)
             return o
-        if tau_batch_stride is None:
-            tau_batch_stride = 0 if tau.dim() == 1 else self.shape.n_q_heads
         decode_sparse(self.shape, self.params, q, k, v, self.meta, n_tokens, tau, tau_batch_stride, o, self.ws,
                       **outs)
         return o
 
     def dense(self, q, k, v, n_tokens: int, tau: Optional[torch.Tensor] = None,
-              tau_batch_stride: Optional[int] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+              tau_batch_stride: Optional[int] = None, out: Optional[torch.Tensor] = None,
+              seq_lens: Optional[torch.Tensor] = None) -> torch.Tensor:
         if tau is not None and tau_batch_stride is None:
             tau_batch_stride = 0 if tau.dim() == 1 else self.shape.n_q_heads
         o = self.out if out is None else out
-        decode_dense(self.shape, self.params, q, k, v, n_tokens, tau, tau_batch_stride or 0, o, self.ws)
+        if seq_lens is not None:
+            decode_dense_ragged(self.shape, self.params, q, k, v, seq_lens, n_tokens, tau, tau_batch_stride or 0, o,
+                                self.ws)
+        else:
+            decode_dense(self.shape, self.params, q, k, v, n_tokens, tau, tau_batch_stride or 0, o, self.ws)
         return o
 
     def device_status(self) -> int:

@@ -121,12 +121,13 @@ eta_status_t check_params(const eta_params_t* p) {
 // fixed shared memory) and index (prefix table and partial counters of B*Hkv
 // entries).
 eta_status_t check_decode_shape(const eta_shape_t* s, bool dense) {
+  (void)dense;  // both passes keep the same segment table
   const int BH = s->batch * s->n_kv_heads;
   if (BH > kMaxBH) return ETA_ERR_UNSUPPORTED;
   const int G = s->n_q_heads / s->n_kv_heads;
   const size_t tile = static_cast<size_t>(s->block_size) * s->head_dim * elem_bytes(s->kv_dtype);
   const size_t fixed = static_cast<size_t>(8) * G * (s->head_dim + 2) * 4 + 16 +
-                       (dense ? 0 : static_cast<size_t>(BH + 1) * 4) + 64;
+                       static_cast<size_t>(BH + 1) * 4 + 64;
   const size_t need = 2 * (2 * tile + 32) + fixed;
   if (need + 1024 > static_cast<size_t>(device_max_smem_optin())) return ETA_ERR_UNSUPPORTED;
   // bf16 K/V with bf16 q take the tensor-core kernel, whose TMA tensor copies
@@ -176,8 +177,9 @@ eta_status_t check_meta(const eta_meta_t& m) {
 eta_status_t do_screen(const eta_shape_t* s, const eta_params_t* p, const void* q, eta_meta_t meta, int64_t n,
                        const float* tau, int64_t tau_stride, const eta_screen_out_t* out, const Workspace& w,
                        cudaStream_t st, const float* W = nullptr, const float* bias = nullptr,
-                       float* tau_out = nullptr) {
+                       float* tau_out = nullptr, const int32_t* seq_lens = nullptr) {
   ScreenCall c;
+  c.seq_lens = seq_lens;
   c.shape = *s;
   c.z = p->z;
   c.offset_a = p->offset_a;
@@ -207,9 +209,9 @@ eta_status_t check_common_decode(const eta_shape_t* s, const eta_params_t* p, co
   return ETA_OK;
 }
 
-eta_status_t do_sparse_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k,
-                              const void* v, int64_t n, const float* tau, int64_t tau_stride, float* out,
-                              const Workspace& w, cudaStream_t st) {
+eta_status_t do_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k, const void* v,
+                       int64_t n, const float* tau, int64_t tau_stride, float* out, const Workspace& w,
+                       cudaStream_t st, bool dense, const int32_t* seq_lens = nullptr) {
   DecodeCall c;
   c.shape = *s;
   c.beta = p->beta;
@@ -217,13 +219,37 @@ eta_status_t do_sparse_decode(const eta_shape_t* s, const eta_params_t* p, const
   c.k = k;
   c.v = v;
   c.n = n;
+  c.seq_lens = seq_lens;
   c.tau = tau;
   c.tau_stride = tau_stride;
   c.out = out;
   c.ws = w;
   c.S = resolve_splits(p);
-  c.dense = false;
+  c.dense = dense;
   return from_cuda(launch_decode(c, st));
+}
+
+eta_status_t do_sparse_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k,
+                              const void* v, int64_t n, const float* tau, int64_t tau_stride, float* out,
+                              const Workspace& w, cudaStream_t st) {
+  return do_decode(s, p, q, k, v, n, tau, tau_stride, out, w, st, false);
+}
+
+eta_status_t check_predictor(const eta_shape_t* s, const void* q, const float* W, const float* bias,
+                             const float* tau);
+
+eta_status_t check_lens(const int32_t* seq_lens) {
+  if (seq_lens == nullptr || !aligned(seq_lens, 4)) return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+// Thresholds of a per-row-length call: given (tau, stride) when W is null,
+// else formed by Eq. 1 into tau_out.
+eta_status_t check_thresholds(const eta_shape_t* s, const void* q, const float* tau, int64_t tau_stride,
+                              const float* W, const float* bias, const float* tau_out) {
+  if (W != nullptr) return check_predictor(s, q, W, bias, tau_out);
+  if (tau == nullptr || tau_stride < 0 || !aligned(tau, 4)) return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
 }
 
 eta_status_t check_predictor(const eta_shape_t* s, const void* q, const float* W, const float* bias,
@@ -370,20 +396,78 @@ ETA_API eta_status_t eta_decode_dense(const eta_shape_t* shape, const eta_params
   if (tau != nullptr && (tau_batch_stride < 0 || !aligned(tau, 4))) return ETA_ERR_INVALID_ARG;
   WsLayout L;
   ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
-  DecodeCall c;
-  c.shape = *shape;
-  c.beta = params->beta;
-  c.q = q;
-  c.k = k;
-  c.v = v;
-  c.n = n_tokens;
-  c.tau = tau;
-  c.tau_stride = tau_batch_stride;
-  c.out = out;
-  c.ws = ws_carve(workspace, L);
-  c.S = resolve_splits(params);
-  c.dense = true;
-  return from_cuda(launch_decode(c, stream));
+  return do_decode(shape, params, q, k, v, n_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L), stream,
+                   true);
+}
+
+ETA_API eta_status_t eta_screen_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                       eta_meta_t meta, const int32_t* seq_lens, int64_t max_tokens,
+                                       const float* tau, int64_t tau_batch_stride, const float* W,
+                                       const float* bias, float* tau_out, const eta_screen_out_t* out,
+                                       void* workspace, size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_shape(shape));
+  ETA_TRY(check_params(params));
+  ETA_TRY(check_tokens(shape, max_tokens));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_screen_shape(shape));
+  ETA_TRY(check_meta(meta));
+  if (q == nullptr || !aligned(q, elem_bytes(shape->q_dtype))) return ETA_ERR_INVALID_ARG;
+  ETA_TRY(check_thresholds(shape, q, tau, tau_batch_stride, W, bias, tau_out));
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_screen(shape, params, q, meta, max_tokens, W ? nullptr : tau, W ? 0 : tau_batch_stride, out,
+                   ws_carve(workspace, L), stream, W, bias, tau_out, seq_lens);
+}
+
+ETA_API eta_status_t eta_decode_sparse_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                              const void* k, const void* v, eta_meta_t meta,
+                                              const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                              int64_t tau_batch_stride, const float* W, const float* bias,
+                                              float* tau_out, float* out, const eta_screen_out_t* extra,
+                                              void* workspace, size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k, v, max_tokens, out));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_screen_shape(shape));
+  ETA_TRY(check_decode_shape(shape, false));
+  ETA_TRY(check_meta(meta));
+  ETA_TRY(check_thresholds(shape, q, tau, tau_batch_stride, W, bias, tau_out));
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  const Workspace w = ws_carve(workspace, L);
+  const float* t = W ? tau_out : tau;
+  const int64_t ts = W ? shape->n_q_heads : tau_batch_stride;
+  ETA_TRY(do_screen(shape, params, q, meta, max_tokens, W ? nullptr : tau, W ? 0 : tau_batch_stride, extra, w,
+                    stream, W, bias, tau_out, seq_lens));
+  return do_decode(shape, params, q, k, v, max_tokens, t, ts, out, w, stream, false, seq_lens);
+}
+
+ETA_API eta_status_t eta_decode_screened_ragged(const eta_shape_t* shape, const eta_params_t* params,
+                                                const void* q, const void* k, const void* v,
+                                                const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                                int64_t tau_batch_stride, float* out, void* workspace,
+                                                size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k, v, max_tokens, out));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_decode_shape(shape, false));
+  if (tau == nullptr || tau_batch_stride < 0 || !aligned(tau, 4)) return ETA_ERR_INVALID_ARG;
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_decode(shape, params, q, k, v, max_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L), stream,
+                   false, seq_lens);
+}
+
+ETA_API eta_status_t eta_decode_dense_ragged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                             const void* k, const void* v, const int32_t* seq_lens,
+                                             int64_t max_tokens, const float* tau, int64_t tau_batch_stride,
+                                             float* out, void* workspace, size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k, v, max_tokens, out));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_decode_shape(shape, true));
+  if (tau != nullptr && (tau_batch_stride < 0 || !aligned(tau, 4))) return ETA_ERR_INVALID_ARG;
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_decode(shape, params, q, k, v, max_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L), stream,
+                   true, seq_lens);
 }
 
 ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t stream, eta_status_t* status) {

@@ -121,6 +121,20 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Cached tokens of batch row b: seq_lens[b] when the call passes per-row
+// lengths (device memory), else the call's uniform count n_max. A length
+// outside [1, n_max] is recorded as ETA_ERR_INVALID_ARG in the status word and
+// clamped, so every kernel of the call sees the same value.
+__device__ __forceinline__ int64_t seq_len_of(const int32_t* seq_lens, int b, int64_t n_max, int32_t* status) {
+  if (seq_lens == nullptr) return n_max;
+  int64_t v = __ldg(seq_lens + b);
+  if (v < 1 || v > n_max) {
+    atomicExch(status, static_cast<int32_t>(ETA_ERR_INVALID_ARG));
+    v = v < 1 ? 1 : n_max;
+  }
+  return v;
+}
+
 // Programmatic dependent launch. The screening and decode kernels are launched
 // with cudaLaunchAttributeProgrammaticStreamSerialization, so each may start
 // (launch, shared-memory and barrier set-up) while the kernel before it on the

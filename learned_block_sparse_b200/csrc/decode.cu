@@ -62,11 +62,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   float* s_mm = s_macc + kNW * G * D;                      // [kNW][G]
   float* s_ml = s_mm + kNW * G;                            // [kNW][G]
   int* s_abort = reinterpret_cast<int*>(s_ml + kNW * G);
-  int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
+  int32_t* s_pre = s_abort + 4;                            // [BH+1] segment starts
 
   grid_dependency_wait();  // inputs may come from the previous kernel on the stream
   allow_dependent_launch();
-  if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kDecThreads);
+  // without per-row lengths a dense pass needs no table: segment i starts at i*nb
+  const bool flat = DENSE && a.seq_lens == nullptr;
+  if (!flat) block_prefix<DENSE>(a, s_pre, BH, kDecThreads);
   if (tid == 0) {
     *s_abort = 0;
     for (int s = 0; s < NST; ++s) {
@@ -78,10 +80,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   __syncthreads();
 
   auto pre = [&](int i) -> int64_t {
-    return DENSE ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
+    return flat ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
   };
   auto seg_of = [&](int64_t p) -> int {
-    return DENSE ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
+    return flat ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
   };
   const int64_t T = pre(BH);
   const int S = gridDim.x;
@@ -112,9 +114,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   float qv[G][VEC], acc[G][VEC], mrun[G], lrun[G], tg[G];
   int cur = seg_of(lo);
   int64_t seg_end = pre(cur + 1);
+  int64_t t_cur = 0;  // position of the current token of segment `cur`
 
   auto load_q = [&](int seg) {
     const int b = seg / a.Hkv, kvh = seg % a.Hkv;
+    t_cur = seg_tokens(a, seg) - 1;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int hq = kvh * G + g;
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
             float v = -INFINITY;
             if (on && r < rows) {
               const float S = sc[jj][g];
-              if (tok0 + r == a.n - 1) {
+              if (tok0 + r == t_cur) {
                 v = S * kLog2e;   // current token: gate exempt (Eq. 3)
               } else {
                 const float x = a.beta * (S - tg[g]);
@@ -276,7 +280,7 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   const int BH = s.batch * s.n_kv_heads;
   const size_t tile = static_cast<size_t>(s.block_size) * D * EB;
   const size_t fixed = static_cast<size_t>(kNW) * G * (D + 2) * sizeof(float) + 16 +
-                       (DENSE ? 0 : static_cast<size_t>(BH + 1) * sizeof(int32_t));
+                       static_cast<size_t>(BH + 1) * sizeof(int32_t);
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
   const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 1024;
   if (fixed + 2 * per_stage > budget) return cudaErrorInvalidValue;

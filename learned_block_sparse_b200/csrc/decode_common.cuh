@@ -19,12 +19,13 @@ struct DecodeArgs {
   const float* tau;
   const uint32_t* union_list;
   const int32_t* union_cnt;
+  const int32_t* seq_lens;  // [B] per-row token counts, or null (every row has n)
   float* o_part;
   float2* ml_part;
   float* out;
   int32_t* seg_done;
   int32_t* status;
-  int64_t cap, n, tau_stride;
+  int64_t cap, n, tau_stride;  // n: tokens of every row, or the upper bound of seq_lens
   int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
   float beta, qscale;
 };
@@ -44,10 +45,18 @@ __device__ __forceinline__ int range_of(int64_t x, int64_t T, int S) {
   return static_cast<int>(((x + 1) * S - 1) / T);
 }
 
-// Exclusive prefix of the union counts into s_pre[0..BH] (all threads call).
-__device__ __forceinline__ void block_prefix(const int32_t* cnt, int32_t* s_pre, int BH, int nthreads) {
+// Cached tokens of segment (batch row, kv head) `seg`.
+__device__ __forceinline__ int64_t seg_tokens(const DecodeArgs& a, int seg) {
+  return seq_len_of(a.seq_lens, seg / a.Hkv, a.n, a.status);
+}
+
+// Exclusive prefix of the per-segment block counts into s_pre[0..BH] (all
+// threads call): the union counts, or (dense) every block of the segment.
+template <bool DENSE>
+__device__ __forceinline__ void block_prefix(const DecodeArgs& a, int32_t* s_pre, int BH, int nthreads) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < BH; i += nthreads) s_pre[i + 1] = cnt[i];
+  for (int i = tid; i < BH; i += nthreads)
+    s_pre[i + 1] = DENSE ? static_cast<int32_t>((seg_tokens(a, i) + a.bs - 1) / a.bs) : a.union_cnt[i];
   __syncthreads();
   if (warp == 0) {
     int run = 0;
@@ -175,28 +184,34 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
   int PL = kMaxPL;  // issuing lanes
   while (PL > NST) PL >>= 1;
   const int lane = threadIdx.x & 31;
-  auto load_entry = [&](int64_t p, int& seg, uint32_t& e) {
+  // entry of position p: segment, (block << 8 | head mask) and the block's
+  // rows (tokens of the row inside the block; -1 when the block is past it)
+  auto load_entry = [&](int64_t p, int& seg, uint32_t& e, int& rows) {
     seg = 0;
     e = 0;
+    rows = 0;
     if (p < hi) {
       seg = seg_of(p);
       const int64_t j = p - pre(seg);
       e = DENSE ? ((static_cast<uint32_t>(j) << 8) | ((1u << G) - 1u))
                 : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + j);
+      const int64_t r = seg_tokens(a, seg) - static_cast<int64_t>(e >> 8) * a.bs;
+      rows = r <= 0 ? -1 : (r < a.bs ? static_cast<int>(r) : a.bs);
     }
   };
-  int seg_cur, seg_nxt = 0;
+  int seg_cur, seg_nxt = 0, rows_cur, rows_nxt = 0;
   uint32_t e_cur, e_nxt = 0;
-  load_entry(lo + lane, seg_cur, e_cur);
+  load_entry(lo + lane, seg_cur, e_cur, rows_cur);
   int issued = 0;    // this lane: 1 + the last position (relative to lo) it armed
   int aborted = 0;
   for (int64_t base = lo; base < hi && !aborted; base += 32) {
-    if (base + 32 < hi) load_entry(base + 32 + lane, seg_nxt, e_nxt);
+    if (base + 32 < hi) load_entry(base + 32 + lane, seg_nxt, e_nxt, rows_nxt);
     const int cnt = static_cast<int>(hi - base < 32 ? hi - base : int64_t{32});
     for (int s = 0; s < cnt && !aborted; s += PL) {
       const int src = s + (lane < PL ? lane : 0);
       const int seg_i = __shfl_sync(kFull, seg_cur, src);
       const uint32_t e_i = __shfl_sync(kFull, e_cur, src);
+      const int rows_i = __shfl_sync(kFull, rows_cur, src);
       if (lane < PL && src < cnt) {
         const int it = static_cast<int>(base - lo) + src;
         const int st = it % NST;
@@ -204,12 +219,10 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
         if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, a.status)) aborted = 1;
         if (!aborted) {
           const int blk = static_cast<int>(e_i >> 8);
-          int rows = 0;
-          if (blk < a.nb) {
-            const int64_t r = a.n - static_cast<int64_t>(blk) * a.bs;
-            rows = r < a.bs ? static_cast<int>(r) : a.bs;
-          } else {
+          int rows = rows_i;
+          if (rows < 0) {  // a list entry past the row's last block: load nothing
             atomicExch(a.status, static_cast<int32_t>(ETA_ERR_INVALID_ARG));
+            rows = 0;
           }
           s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
           if (rows == 0) mbar_arrive(&s_full[st]);
@@ -221,6 +234,7 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
     }
     seg_cur = seg_nxt;
     e_cur = e_nxt;
+    rows_cur = rows_nxt;
   }
   if (aborted && lane < PL) {
     // let the copies this lane armed land before the thread block can exit
@@ -249,6 +263,7 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.status = c.ws.status;
   a.cap = s.capacity;
   a.n = c.n;
+  a.seq_lens = c.seq_lens;
   a.tau_stride = c.tau_stride;
   a.B = s.batch;
   a.Hq = s.n_q_heads;

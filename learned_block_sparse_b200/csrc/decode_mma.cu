@@ -137,11 +137,13 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   float* s_mm = s_macc + kMW * G * D;                      // [kMW][G]
   float* s_ml = s_mm + kMW * G;                            // [kMW][G]
   int* s_abort = reinterpret_cast<int*>(s_ml + kMW * G);
-  int32_t* s_pre = s_abort + 4;                            // [BH+1] (sparse only)
+  int32_t* s_pre = s_abort + 4;                            // [BH+1] segment starts
 
   grid_dependency_wait();  // inputs may come from the previous kernel on the stream
   allow_dependent_launch();
-  if (!DENSE) block_prefix(a.union_cnt, s_pre, BH, kMmaThreads);
+  // without per-row lengths a dense pass needs no table: segment i starts at i*nb
+  const bool flat = DENSE && a.seq_lens == nullptr;
+  if (!flat) block_prefix<DENSE>(a, s_pre, BH, kMmaThreads);
   if (tid == 0) {
     *s_abort = 0;
     for (int s = 0; s < NST; ++s) {
@@ -153,10 +155,10 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   __syncthreads();
 
   auto pre = [&](int i) -> int64_t {
-    return DENSE ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
+    return flat ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
   };
   auto seg_of = [&](int64_t p) -> int {
-    return DENSE ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
+    return flat ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
   };
   const int64_t T = pre(BH);
   const int S = gridDim.x;
@@ -191,9 +193,11 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   uint32_t qa[KST][2];
   float o[NDT][4];  // [n-tile][c0 c1 = high part of row, c2 c3 = low part]
   float m_r = -INFINITY, l_r = 0.0f, tau_r = 0.0f;
+  int64_t t_cur = 0;  // position of the current token of the segment being attended
 
   auto load_q = [&](int seg) {
     const int b = seg / a.Hkv, kvh = seg % a.Hkv;
+    t_cur = seg_tokens(a, seg) - 1;
     if (live_row) {
       const uint16_t* qp =
           static_cast<const uint16_t*>(a.q) + (static_cast<int64_t>(b) * a.Hq + kvh * G + row) * D;
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     const bool row_on = live_row && ((static_cast<uint32_t>(inf.y) >> row) & 1u);
     const int64_t tok0 = static_cast<int64_t>(inf.x) * bs;
     // full block that does not hold the current token: no per-key checks
-    const bool fast = rows == bs && tok0 + bs <= a.n - 1;
+    const bool fast = rows == bs && tok0 + bs <= t_cur;
     constexpr int NT = CH / 8;  // n-tiles of 8 keys per chunk
     for (int c0 = 0; c0 < bs; c0 += CH) {
       // S = Q K^T: even and odd k-steps accumulate separately (shorter mma chains)
@@ -286,7 +290,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
             if (row_on && key < rows) {
               const float Sv = (se[j][e] + so[j][e]) * a.qscale;
               // the current token is exempt from the gate (Eq. 3)
-              v = (tok0 + key == a.n - 1) ? Sv * kLog2e : gate(Sv);
+              v = (tok0 + key == t_cur) ? Sv * kLog2e : gate(Sv);
             }
             g[j][e] = v;
             bm = fmaxf(bm, v);
@@ -416,7 +420,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
   constexpr int kMW = MmaWarps<D, CH>::kMW;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 +
-                       (DENSE ? 0 : static_cast<size_t>(BH + 1) * sizeof(int32_t)) + 1024;
+                       static_cast<size_t>(BH + 1) * sizeof(int32_t) + 1024;
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
   const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 512;
   if (fixed + 2 * per_stage > budget) return cudaErrorInvalidValue;

@@ -83,7 +83,8 @@ struct ScreenCall {
   int n_local;
   const void* q;
   eta_meta_t meta;
-  int64_t n;
+  int64_t n;               // tokens (all rows), or the upper bound of seq_lens
+  const int32_t* seq_lens; // [B] per-row token counts (device), or null
   const float* tau;
   int64_t tau_stride;
   const float* W;         // non-null: form tau by Eq. 1 inside the screen (tau ignored)
@@ -100,7 +101,8 @@ struct DecodeCall {
   const void* q;
   const void* k;
   const void* v;
-  int64_t n;
+  int64_t n;               // tokens (all rows), or the upper bound of seq_lens
+  const int32_t* seq_lens; // [B] per-row token counts (device), or null
   const float* tau;        // gate thresholds; null = -inf (dense only)
   int64_t tau_stride;
   float* out;

@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
   allow_dependent_launch();
   screen_prologue<D, G, 32, true>(a, sm, b, kvh, kScreenWarps * 32);
 
-  const int nt = (a.ns + 31) / 32;
+  const RowBlocks rb = row_blocks(a, b);
+  const int nt = (rb.ns + 31) / 32;
   const int t0 = cr * tpc;
   const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
   const float* mu = a.mu + static_cast<int64_t>(bh) * D * a.nb_cap;
@@ -54,8 +55,8 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
 #pragma unroll
     for (int u = 0; u < kSub; ++u) {
       const int blk = (t0 + t4 + u) * 32 + lane;
-      valid[u] = (t4 + u < my_tiles) && blk < a.ns;
-      cb[u] = blk < a.ns ? blk : a.ns - 1;
+      valid[u] = (t4 + u < my_tiles) && blk < rb.ns;
+      cb[u] = blk < rb.ns ? blk : rb.ns - 1;  // rb.ns >= 1 here (this warp has a tile)
     }
     float dg[kSub][G], vg[kSub][G];
 #pragma unroll
@@ -90,7 +91,7 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
     }
   }
   __syncthreads();
-  screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, kScreenWarps * 32);
+  screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, rb, kScreenWarps * 32);
 }
 
 template <int D, int G>

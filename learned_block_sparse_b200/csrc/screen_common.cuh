@@ -26,7 +26,11 @@ struct ScreenArgs {
   const float* bias;
   float* tau_out;
   float z, s, offset_a;
-  int Hq, Hkv, nb, ns, nb_cap, tiles_per_cta;
+  int Hq, Hkv, nb, ns, nb_cap, tiles_per_cta;  // nb, ns: of the longest row (launch sizing)
+  const int32_t* seq_lens;  // [B] per-row token counts, or null (every row has n)
+  int64_t n;
+  int bs, n_local;
+  int32_t* status;
   uint32_t* ws_union;
   int32_t* ws_union_cnt;
   int32_t* ws_head_cnt;
@@ -35,6 +39,12 @@ struct ScreenArgs {
   uint32_t* union_out;
   int32_t* union_cnt_out;
   float* scores;
+};
+
+// Blocks of batch row b: nb in all, the first ns of them screened (the last
+// n_local, which hold the current token, are always admitted).
+struct RowBlocks {
+  int nb, ns;
 };
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
@@ -75,6 +85,14 @@ struct ScreenSmem {
     return fixed_bytes() + static_cast<size_t>(tpc) * (G + 1) * sizeof(int) + static_cast<size_t>(tpc) * 32;
   }
 };
+
+__device__ __forceinline__ RowBlocks row_blocks(const ScreenArgs& a, int b) {
+  const int64_t n = seq_len_of(a.seq_lens, b, a.n, a.status);
+  RowBlocks r;
+  r.nb = static_cast<int>((n + a.bs - 1) / a.bs);
+  r.ns = max(0, r.nb - a.n_local);
+  return r;
+}
 
 // Eq. 1 thresholds of the group's heads (a.W set) by the `nthreads` threads
 // with relative index `rel`, synchronised by `sync`: sm.tau, sm.taut = tau - a,
@@ -172,7 +190,7 @@ __device__ __forceinline__ void screen_record_tile(const ScreenSmem<D, G>& sm, i
 // the counts.
 template <int D, int G>
 __device__ __forceinline__ void screen_finish(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
-                                              int bh, int t0, int my_tiles, int nthreads) {
+                                              int bh, int t0, int my_tiles, RowBlocks rb, int nthreads) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = static_cast<int>(cluster.num_blocks());
@@ -219,10 +237,10 @@ __device__ __forceinline__ void screen_finish(const ScreenArgs& a, const ScreenS
   }
 
   if (cr == cs - 1) {
-    const int nf = a.nb - a.ns;
+    const int nf = rb.nb - rb.ns;
     const uint32_t all = (1u << G) - 1u;
     for (int j = tid; j < nf; j += nthreads) {
-      const int blk = a.ns + j;
+      const int blk = rb.ns + j;
       if (a.active_idx != nullptr) {
 #pragma unroll
         for (int g = 0; g < G; ++g)
@@ -267,6 +285,11 @@ inline ScreenArgs make_screen_args(const ScreenCall& c, int nb, int ns, int tpc)
   a.Hkv = s.n_kv_heads;
   a.nb = nb;
   a.ns = ns;
+  a.seq_lens = c.seq_lens;
+  a.n = c.n;
+  a.bs = s.block_size;
+  a.n_local = c.n_local;
+  a.status = c.ws.status;
   a.nb_cap = static_cast<int>(s.capacity / s.block_size);
   a.tiles_per_cta = tpc;
   a.ws_union = c.ws.union_list;

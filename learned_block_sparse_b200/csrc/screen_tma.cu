@@ -75,9 +75,6 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   static_assert((static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>) % 16 == 0, "ScreenSmem alignment");
   const ScreenSmem<D, G> sm(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>, tpc);
 
-  const int nt = (a.ns + 31) / 32;
-  const int t0 = cr * tpc;
-  const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
   const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
 
   if (tid == 0) {
@@ -91,6 +88,10 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   }
   grid_dependency_wait();  // inputs may come from the previous kernel on the stream
   allow_dependent_launch();
+  const RowBlocks rb = row_blocks(a, b);
+  const int nt = (rb.ns + 31) / 32;
+  const int t0 = cr * tpc;
+  const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
   __syncthreads();
   auto issue_tile = [&](int it) {
     const int st = it % NST;
@@ -144,8 +145,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
     for (int it = warp; it < my_tiles; it += CW) {
       const int st = it % NST;
       const int blk = (t0 + it) * 32 + lane;
-      const bool valid = blk < a.ns;
-      const float M = __ldg(mx + (valid ? blk : a.ns - 1));
+      const bool valid = blk < rb.ns;
+      const float M = __ldg(mx + (valid ? blk : rb.ns - 1));  // rb.ns >= 1 here (this CTA has a tile)
       const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status);
       float dg[G], vg[G];
 #pragma unroll
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
     }
   }
   __syncthreads();
-  screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, NT);
+  screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, rb, NT);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 meta_map_encoder() {
