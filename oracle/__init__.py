@@ -61,7 +61,7 @@ def lib():
         L.oracle_inv_sqrt_d.restype = f32
         L.oracle_screen_head.argtypes = [vp, i32, vp, vp, vp, i64, i32, f32, f32, f32, vp, vp]
         L.oracle_screen_head.restype = i32
-        L.oracle_attend_head.argtypes = [i32, vp, vp, i32, i32, i64, vp, vp, i32, f32, f32, vp]
+        L.oracle_attend_head.argtypes = [i32, vp, vp, i32, i32, i64, vp, vp, i32, f32, f32, i32, vp]
         for fn in ("oracle_to_f32", "oracle_block_meta", "oracle_slice_meta",
                    "oracle_predict_tau", "oracle_attend_head"):
             getattr(L, fn).restype = None
@@ -182,9 +182,15 @@ def screen_head(q_f32, mu, var, maxn, nb: int, n_local: int, z: float, tau: floa
     return lst[:cnt].copy(), sc[:ns].copy()
 
 
+GATE_SIGMOID, GATE_HARD = 0, 1
+
+
 def attend_head(k_slice, v_slice, bs: int, n: int, q_f32, blocks, tau: float,
-                beta: float) -> np.ndarray:
-    """Gated softmax attention (Eq. 2-3) of one head over the listed blocks -> [d] float64."""
+                beta: float, gate: int = GATE_SIGMOID) -> np.ndarray:
+    """Gated softmax attention of one head over the listed blocks -> [d] float64.
+    gate GATE_SIGMOID: Eq. 2-3 (multiplicative gate, the pages' normal mode);
+    GATE_HARD: keys below tau removed (strict mode, Tables 6-7); the current
+    token is exempt in both."""
     ka, dt = _raw(k_slice)
     va, dt2 = _raw(v_slice)
     assert dt == dt2
@@ -193,7 +199,7 @@ def attend_head(k_slice, v_slice, bs: int, n: int, q_f32, blocks, tau: float,
     blocks = np.ascontiguousarray(blocks, np.int32)
     out = np.zeros((d,), np.float64)
     lib().oracle_attend_head(dt, _p(ka), _p(va), d, bs, n, _p(q_f32), _p(blocks),
-                             int(blocks.size), float(tau), float(beta), _p(out))
+                             int(blocks.size), float(tau), float(beta), int(gate), _p(out))
     return out
 
 

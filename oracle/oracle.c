@@ -169,13 +169,16 @@ static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
  * Methodology §2, Eq. 2-3, restricted to the loaded blocks (Figure 6):
  *   S_s = <q, k_s> / sqrt(d)
  *   g_s = S_s                                  if s = t (the current token, t = n-1)
- *   g_s = S_s * sigma(beta * (S_s - tau))      otherwise
+ *   g_s = S_s * sigma(beta * (S_s - tau))      otherwise (gate 0: the multiplicative
+ *                                              gate, the pages' "normal mode")
+ *   g_s = S_s if S_s >= tau, else -infinity    otherwise (gate 1: "strict mode", hard
+ *                                              additive masking, Tables 6-7)
  *   o   = sum_s exp(g_s - max g) v_s / sum_s exp(g_s - max g)
  * over every token s < n of every listed block.
  *   k, v : slice [cap][d] in kv_dtype;  q : [d] fp32 values;  out : [d]
  */
 void oracle_attend_head(int kv_dtype, const void* k, const void* v, int d, int bs, int64_t n,
-                        const float* q, const int32_t* list, int cnt, float tau, float beta,
+                        const float* q, const int32_t* list, int cnt, float tau, float beta, int gate,
                         double* out) {
   const double inv = 1.0 / sqrt((double)d);
   const int64_t t = n - 1;
@@ -190,7 +193,10 @@ void oracle_attend_head(int kv_dtype, const void* k, const void* v, int d, int b
       double S = 0.0;
       for (int i = 0; i < d; ++i) S += (double)q[i] * (double)elem(k, kv_dtype, s * d + i);
       S *= inv;
-      double gs = (s == t) ? S : S * sigmoid((double)beta * (S - (double)tau));
+      double gs;
+      if (s == t) gs = S;                                   /* Eq. 3: the current token is exempt */
+      else if (gate == 0) gs = S * sigmoid((double)beta * (S - (double)tau));   /* Eq. 2 */
+      else gs = (S >= (double)tau) ? S : -INFINITY;         /* strict mode: hard mask */
       g[m] = gs;
       pos[m] = s;
       if (gs > gmax) gmax = gs;

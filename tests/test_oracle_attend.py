@@ -121,3 +121,72 @@ def test_full_decode_gqa_union_is_or_of_heads():
     vv = V[1, 5 // w.G, :w.n].double()
     ref = torch.softmax(kk @ qf / math.sqrt(w.d), 0) @ vv
     assert np.allclose(resd["out"][(1, 5)], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------- strict mode (hard masking)
+def test_hard_gate_minus_inf_is_softmax_attention():
+    """Strict mode with tau = -inf removes nothing: textbook softmax attention."""
+    n, bs, d = 150, 16, 64
+    rng = np.random.default_rng(11)
+    k, v = _kv(rng, n, d, bs)
+    q = rng.standard_normal(d).astype(np.float32)
+    nb = (n + bs - 1) // bs
+    out = oracle.attend_head(k, v, bs, n, q, np.arange(nb, dtype=np.int32), float("-inf"), 5.0,
+                             gate=oracle.GATE_HARD)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).double()[None, None, None, :],
+        torch.from_numpy(k[:n]).double()[None, None], torch.from_numpy(v[:n]).double()[None, None])
+    assert np.allclose(out, ref[0, 0, 0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_hard_gate_plus_inf_keeps_only_the_current_token():
+    """Every key but the current one is removed: the output is v_t exactly
+    (where the multiplicative gate leaves the uniform floor instead)."""
+    n, bs, d = 77, 16, 64
+    rng = np.random.default_rng(12)
+    k, v = _kv(rng, n, d, bs)
+    q = rng.standard_normal(d).astype(np.float32)
+    nb = (n + bs - 1) // bs
+    out = oracle.attend_head(k, v, bs, n, q, np.arange(nb, dtype=np.int32), float("inf"), 5.0,
+                             gate=oracle.GATE_HARD)
+    assert np.array_equal(out, v[n - 1].astype(np.float64))
+
+
+@pytest.mark.parametrize("quantile", [0.3, 0.8, 0.97])
+def test_hard_gate_equals_softmax_over_the_kept_keys(quantile):
+    """Strict mode over a cache equals the plain softmax (tau = -inf) of the oracle
+    over a second cache holding only the keys with S >= tau and the current token,
+    in order: removing a key and masking it to -inf must agree. The kept set is
+    chosen by numpy in float64, independently of the oracle's comparison."""
+    n, bs, d = 300, 16, 64
+    rng = np.random.default_rng(int(quantile * 100))
+    k, v = _kv(rng, n, d, bs)
+    q = rng.standard_normal(d).astype(np.float32)
+    S = (k[:n].astype(np.float64) @ q.astype(np.float64)) / math.sqrt(d)
+    tau = float(np.quantile(S, quantile)) + 1e-6
+    nb = (n + bs - 1) // bs
+    out = oracle.attend_head(k, v, bs, n, q, np.arange(nb, dtype=np.int32), tau, 5.0, gate=oracle.GATE_HARD)
+    keep = np.nonzero(S >= tau)[0].tolist()
+    if n - 1 not in keep:
+        keep.append(n - 1)
+    m = len(keep)
+    k2, v2 = _kv(rng, m, d, bs)
+    k2[:m], v2[:m] = k[keep], v[keep]
+    nb2 = (m + bs - 1) // bs
+    ref = oracle.attend_head(k2, v2, bs, m, q, np.arange(nb2, dtype=np.int32), float("-inf"), 5.0)
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_hard_gate_keeps_a_key_exactly_at_the_threshold():
+    """S == tau is kept (the comparison is >=, as the screen's admission rule)."""
+    d, bs = 4, 16
+    k = np.zeros((16, d), np.float32)
+    v = np.zeros((16, d), np.float32)
+    k[0] = [2, 0, 0, 0]            # S_0 = 1
+    k[1] = [1.0, 0, 0, 0]          # S_1 = 0.5 < tau: removed
+    k[2] = [0, 0, 0, 0]            # current token, S_t = 0
+    v[0], v[1], v[2] = [1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0]
+    q = np.array([1, 0, 0, 0], np.float32)
+    out = oracle.attend_head(k, v, bs, 3, q, np.array([0], np.int32), 1.0, 5.0, gate=oracle.GATE_HARD)
+    e = math.e
+    assert np.allclose(out, [e / (e + 1), 0, 1 / (e + 1), 0], rtol=1e-14)
