@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define ETA_ABI_VERSION 1
+#define ETA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define ETA_API __attribute__((visibility("default")))
@@ -89,7 +89,16 @@ typedef struct {
                           last block holds the current token, whose gate Eq. 3
                           exempts) */
   int32_t n_splits;    /* decode work ranges (thread blocks); 0 = one per SM */
+  int32_t gate;        /* ETA_GATE_SIGMOID (Eq. 2-3) or ETA_GATE_HARD (strict mode) */
 } eta_params_t;
+
+/* Logit gate of the decode (the current token t is exempt from both):
+ * ETA_GATE_SIGMOID  g_s = S_s * sigmoid(beta (S_s - tau))   (Eq. 2-3; the pages'
+ *                   "normal mode", multiplicative gating)
+ * ETA_GATE_HARD     g_s = S_s if S_s >= tau, else -infinity: keys below the
+ *                   threshold are removed (the "strict mode" of Tables 6-7,
+ *                   hard additive masking; beta unused) */
+enum { ETA_GATE_SIGMOID = 0, ETA_GATE_HARD = 1 };
 
 /* Block metadata of Methodology §4 ("Dual Probabilistic-Geometric Block
  * Index"): population centroid, coordinate-wise population variance and

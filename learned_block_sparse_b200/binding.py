@@ -33,9 +33,12 @@ class Shape(ctypes.Structure):
                 ("kv_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32)]
 
 
+GATE_SIGMOID, GATE_HARD = 0, 1   # Eq. 2-3 multiplicative gate; strict mode (hard masking)
+
+
 class Params(ctypes.Structure):
     _fields_ = [("beta", ctypes.c_float), ("z", ctypes.c_float), ("offset_a", ctypes.c_float),
-                ("n_local", ctypes.c_int32), ("n_splits", ctypes.c_int32)]
+                ("n_local", ctypes.c_int32), ("n_splits", ctypes.c_int32), ("gate", ctypes.c_int32)]
 
 
 class Meta(ctypes.Structure):
@@ -138,8 +141,8 @@ def make_shape(batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity, kv_
                  _dtype_code(q_dtype) if isinstance(q_dtype, torch.dtype) else q_dtype)
 
 
-def make_params(beta=5.0, z=1.0, offset_a=0.0, n_local=1, n_splits=0) -> Params:
-    return Params(beta, z, offset_a, n_local, n_splits)
+def make_params(beta=5.0, z=1.0, offset_a=0.0, n_local=1, n_splits=0, gate=GATE_SIGMOID) -> Params:
+    return Params(beta, z, offset_a, n_local, n_splits, gate)
 
 
 def build_block_meta(shape: Shape, k: torch.Tensor, blk_begin: int, blk_end: int, mu: torch.Tensor,
@@ -299,9 +302,9 @@ class EtaDecoder:
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity,
                  kv_dtype=torch.bfloat16, q_dtype=torch.bfloat16, beta=5.0, z=1.0, offset_a=0.0,
-                 n_local=1, n_splits=0, device="cuda"):
+                 n_local=1, n_splits=0, device="cuda", gate=GATE_SIGMOID):
         self.shape = make_shape(batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity, kv_dtype, q_dtype)
-        self.params = make_params(beta, z, offset_a, n_local, n_splits)
+        self.params = make_params(beta, z, offset_a, n_local, n_splits, gate)
         self.device = torch.device(device)
         nb_cap = capacity // block_size
         f = dict(dtype=torch.float32, device=self.device)

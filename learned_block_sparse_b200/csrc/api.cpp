@@ -114,6 +114,7 @@ eta_status_t check_params(const eta_params_t* p) {
   if (!(p->beta > 0.0f) || !std::isfinite(p->beta)) return ETA_ERR_INVALID_ARG;
   if (!std::isfinite(p->z) || !std::isfinite(p->offset_a)) return ETA_ERR_INVALID_ARG;
   if (p->n_local < 1 || p->n_splits < 0) return ETA_ERR_INVALID_ARG;
+  if (p->gate != ETA_GATE_SIGMOID && p->gate != ETA_GATE_HARD) return ETA_ERR_INVALID_ARG;
   return ETA_OK;
 }
 
@@ -215,6 +216,7 @@ eta_status_t do_decode(const eta_shape_t* s, const eta_params_t* p, const void* 
   DecodeCall c;
   c.shape = *s;
   c.beta = p->beta;
+  c.gate = p->gate;
   c.q = q;
   c.k = k;
   c.v = v;

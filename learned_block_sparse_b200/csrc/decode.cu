@@ -183,6 +183,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
               const float S = sc[jj][g];
               if (tok0 + r == t_cur) {
                 v = S * kLog2e;   // current token: gate exempt (Eq. 3)
+              } else if (a.gate == ETA_GATE_HARD) {
+                v = S >= tg[g] ? S * kLog2e : -INFINITY;   // strict mode: removed below tau
               } else {
                 const float x = a.beta * (S - tg[g]);
                 const float sig = __frcp_rn(1.0f + exp2f(-x * kLog2e));

@@ -27,6 +27,7 @@ struct DecodeArgs {
   int32_t* status;
   int64_t cap, n, tau_stride;  // n: tokens of every row, or the upper bound of seq_lens
   int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
+  int gate;  // ETA_GATE_SIGMOID or ETA_GATE_HARD
   float beta, qscale;
 };
 
@@ -274,6 +275,7 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.nstages = nstages;
   a.q_dtype = s.q_dtype;
   a.beta = c.beta;
+  a.gate = c.gate;
   a.qscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.head_dim)));
   return a;
 }

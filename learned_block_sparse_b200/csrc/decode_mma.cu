@@ -111,7 +111,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-template <int D, int G, bool DENSE, int CH>
+// HARD: the strict-mode gate (keys below tau removed) instead of Eq. 2-3.
+template <int D, int G, bool DENSE, int CH, bool HARD>
 __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
@@ -237,9 +238,13 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     finish_segment<D, G, kMW>(a, seg, pre(seg), pre(seg + 1), lo, T, S, s_macc, s_mm, s_ml, s_abort + 1);
   };
 
-  // gate in log2 units: g = S * sigmoid(beta (S - tau)) * log2(e)
+  // gate in log2 units: g = S * sigmoid(beta (S - tau)) * log2(e), or (strict
+  // mode) S * log2(e) for S >= tau and -inf below
   const float nbl = -a.beta * kLog2e;
-  auto gate = [&](float Sv) { return Sv * rcp_approx(1.0f + ex2_approx(nbl * (Sv - tau_r))) * kLog2e; };
+  auto gate = [&](float Sv) {
+    if (HARD) return Sv >= tau_r ? Sv * kLog2e : -INFINITY;
+    return Sv * rcp_approx(1.0f + ex2_approx(nbl * (Sv - tau_r))) * kLog2e;
+  };
 
   auto process = [&](int st, const int4 inf) {
     const uint32_t kt = smem_u32(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes);
@@ -438,12 +443,19 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size))
     return cudaErrorInvalidValue;
 
-  static std::atomic<uint64_t> smem_done{0};
-  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH>));
-  if (e != cudaSuccess) return e;
   const DecodeArgs a = make_decode_args(c, nst);
-  return launch_pdl(decode_mma_kernel<D, G, DENSE, CH>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads, smem,
-                    st, a, tmk, tmv);
+  if (c.gate == ETA_GATE_HARD) {
+    static std::atomic<uint64_t> smem_done{0};
+    cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, true>));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, true>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads,
+                      smem, st, a, tmk, tmv);
+  }
+  static std::atomic<uint64_t> smem_done{0};
+  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, false>));
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, false>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads,
+                    smem, st, a, tmk, tmv);
 }
 
 template <int D, bool DENSE, int CH>

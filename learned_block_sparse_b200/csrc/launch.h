@@ -98,6 +98,7 @@ cudaError_t launch_screen(const ScreenCall& c, cudaStream_t st);
 struct DecodeCall {
   eta_shape_t shape;
   float beta;
+  int gate;                // ETA_GATE_SIGMOID or ETA_GATE_HARD
   const void* q;
   const void* k;
   const void* v;

@@ -106,7 +106,8 @@ def run_gpu(dw, tau, stride, bias=None, dense=False):
     return res
 
 
-def oracle_step(w, q_host, K_host, V_host, meta, tau, stride, heads, dense=False, offset_a=0.0):
+def oracle_step(w, q_host, K_host, V_host, meta, tau, stride, heads, dense=False, offset_a=0.0,
+                gate=oracle.GATE_SIGMOID):
     qf = oracle.to_f32(q_host)
     tau_arr = np.asarray(tau, np.float32)
 
@@ -121,7 +122,7 @@ def oracle_step(w, q_host, K_host, V_host, meta, tau, stride, heads, dense=False
             mu, var, mx = meta[(b, kvh)]
             lst, sc = oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, tau_of(b, hq), offset_a)
         t_gate = float("-inf") if (dense and tau is None) else tau_of(b, hq)
-        o = oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, w.n, qf[b, hq], lst, t_gate, w.beta)
+        o = oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, w.n, qf[b, hq], lst, t_gate, w.beta, gate)
         return (b, hq), (lst, sc, o)
     return dict(pmap(one, heads))
 

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     from learned_block_sparse_b200 import binding
-    assert binding.lib.eta_abi_version() == 1
+    assert binding.lib.eta_abi_version() == 2
     assert binding.status_string(0) == "ok"
     assert "workspace" in binding.status_string(3)
     assert binding.status_string(99) == "unknown status"
@@ -91,9 +91,16 @@ def test_argument_validation_before_launch():
                                a16, 64, None) == 3
     # params
     for bad_p in (binding.make_params(beta=0.0), binding.make_params(n_local=0), binding.make_params(n_splits=-1),
-                  binding.make_params(z=float("nan"))):
+                  binding.make_params(z=float("nan")), binding.make_params(gate=2)):
         assert L.eta_decode_dense(ctypes.byref(s), ctypes.byref(bad_p), a16, a16, a16, 100, None, 0, a16, a16,
                                   1 << 30, None) == 1
+    # per-row lengths: the length array is required; max_tokens bounded by the capacity
+    assert L.eta_decode_dense_ragged(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, None, 100, None, 0, a16,
+                                     a16, 1 << 30, None) == 1
+    assert L.eta_decode_dense_ragged(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, a16, s.capacity + 1, None, 0,
+                                     a16, a16, 1 << 30, None) == 1
+    assert L.eta_decode_sparse_ragged(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, a16, 100, None, 0,
+                                      None, None, None, a16, None, a16, 1 << 30, None) == 1   # no thresholds
     # metadata block range
     assert L.eta_build_block_meta(ctypes.byref(s), a16, -1, 3, meta, None) == 1
     assert L.eta_build_block_meta(ctypes.byref(s), a16, 0, 33, meta, None) == 1

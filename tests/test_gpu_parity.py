@@ -249,6 +249,33 @@ def test_thresholds_in_screen_equal_separate_predictor(dtype, G, bs):
     assert torch.equal(fused, sep)
 
 
+@pytest.mark.parametrize("dtype,G,bs", [("bf16", 4, 32), ("bf16", 8, 64), ("f32", 1, 16), ("bf16", 1, 16)])
+def test_strict_mode_gate(dtype, G, bs):
+    """Strict mode (keys below tau removed): lists and outputs against the oracle.
+    Each head's tau sits in a wide gap of its own true logits, so the keep/remove
+    decision does not depend on how either side rounds S."""
+    d = 64 if (G == 8 or dtype == "f32") else 128
+    w = synth.Workload("strict", dtype, 2, 2 * G, 2, d, bs * 60 + 5, bs, z=1.0, tau_mode="const",
+                       densities=(0.5,), seed=300 + G + bs, offset_std=synth.SQRT_HALF)
+    dw = DeviceWorkload(w, keep_host=True, gate=binding.GATE_HARD)
+    meta = parity.oracle_meta(w, dw.K_host)
+    qf = oracle.to_f32(dw.q_host).astype(np.float64)
+    tau = np.zeros((w.B, w.Hq), np.float32)
+    for b in range(w.B):
+        for h in range(w.Hq):
+            k = dw.K_host[b, h // w.G, :w.n].double().numpy()
+            S = np.sort(k @ qf[b, h] / math.sqrt(w.d))
+            i0 = int(0.85 * w.n)
+            i = max(range(i0 - 40, i0 + 40), key=lambda j: S[j + 1] - S[j])
+            assert S[i + 1] - S[i] > 1e-4
+            tau[b, h] = np.float32(0.5 * (S[i] + S[i + 1]))
+    gpu = parity.run_gpu(dw, tau, w.Hq)
+    assert gpu["status"] == 0
+    heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, w.Hq, heads, gate=oracle.GATE_HARD)
+    parity.compare(w, gpu, orc, heads)
+
+
 # ----------------------------------------------------------------- full size
 def _sample_heads(w, k, seed=0):
     rng = np.random.default_rng(seed)
