@@ -100,6 +100,18 @@ typedef struct {
  *                   hard additive masking; beta unused) */
 enum { ETA_GATE_SIGMOID = 0, ETA_GATE_HARD = 1 };
 
+/* A paged KV store: the K and V pools are [num_pages][Hkv][block_size][d]
+ * (one page holds one block of every kv head) and row b's logical block j
+ * lives in page block_table[b * (capacity / block_size) + j]. capacity is the
+ * logical capacity of a row. A page index outside [0, num_pages) is never
+ * read: the block is skipped and ETA_ERR_INVALID_ARG is recorded in the
+ * device status word (by the decode; the metadata build leaves the block's
+ * metadata as it was). */
+typedef struct {
+  const int32_t* block_table;  /* [B][capacity / block_size] int32, device memory */
+  int32_t num_pages;
+} eta_pages_t;
+
 /* Block metadata of Methodology §4 ("Dual Probabilistic-Geometric Block
  * Index"): population centroid, coordinate-wise population variance and
  * maximum key norm of each full block. Layout in the conventions above. */
@@ -302,6 +314,35 @@ ETA_API eta_status_t eta_decode_dense_ragged(const eta_shape_t* shape, const eta
                                              const void* k, const void* v, const int32_t* seq_lens,
                                              int64_t max_tokens, const float* tau, int64_t tau_batch_stride,
                                              float* out, void* workspace, size_t ws_bytes, eta_stream_t stream);
+
+/*
+ * Paged KV (see eta_pages_t): the per-row-length calls on K and V pools
+ * addressed through a block table, with per-row lengths (seq_lens,
+ * max_tokens) as in eta_decode_sparse_ragged. The metadata stays indexed by
+ * logical block ([B][Hkv][d][capacity / block_size]); eta_build_block_meta_paged
+ * builds it from the pool. A row's result equals the contiguous call on the
+ * cache its pages describe, bit for bit.
+ */
+ETA_API eta_status_t eta_build_block_meta_paged(const eta_shape_t* shape, const void* k_pool, eta_pages_t pages,
+                                                int64_t blk_begin, int64_t blk_end, eta_meta_t meta,
+                                                eta_stream_t stream);
+ETA_API eta_status_t eta_decode_sparse_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                             const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                             eta_meta_t meta, const int32_t* seq_lens, int64_t max_tokens,
+                                             const float* tau, int64_t tau_batch_stride, const float* W,
+                                             const float* bias, float* tau_out, float* out,
+                                             const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
+                                             eta_stream_t stream);
+ETA_API eta_status_t eta_decode_screened_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                               const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                               const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                               int64_t tau_batch_stride, float* out, void* workspace,
+                                               size_t ws_bytes, eta_stream_t stream);
+ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                            const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                            const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                            int64_t tau_batch_stride, float* out, void* workspace, size_t ws_bytes,
+                                            eta_stream_t stream);
 
 /*
  * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and

@@ -45,6 +45,10 @@ class Meta(ctypes.Structure):
     _fields_ = [("mu", ctypes.c_void_p), ("var", ctypes.c_void_p), ("maxnorm", ctypes.c_void_p)]
 
 
+class Pages(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int32)]
+
+
 class ScreenOut(ctypes.Structure):
     _fields_ = [("active_idx", ctypes.c_void_p), ("active_cnt", ctypes.c_void_p),
                 ("union_list", ctypes.c_void_p), ("union_cnt", ctypes.c_void_p), ("scores", ctypes.c_void_p)]
@@ -88,6 +92,15 @@ def _load():
     L.eta_decode_screened_ragged.argtypes = [P(Shape), P(Params), vp, vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense_ragged.restype = st
     L.eta_decode_dense_ragged.argtypes = [P(Shape), P(Params), vp, vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
+    L.eta_build_block_meta_paged.restype = st
+    L.eta_build_block_meta_paged.argtypes = [P(Shape), vp, Pages, i64, i64, Meta, vp]
+    L.eta_decode_sparse_paged.restype = st
+    L.eta_decode_sparse_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, Meta, vp, i64, vp, i64, vp, vp, vp,
+                                          vp, P(ScreenOut), vp, sz, vp]
+    L.eta_decode_screened_paged.restype = st
+    L.eta_decode_screened_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
+    L.eta_decode_dense_paged.restype = st
+    L.eta_decode_dense_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_screened.restype = st
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
@@ -105,7 +118,8 @@ EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta
             "eta_decode_workspace_bytes", "eta_workspace_init", "eta_screen", "eta_decode_sparse",
             "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static",
             "eta_screen_predict", "eta_decode_sparse_predict", "eta_screen_ragged", "eta_decode_sparse_ragged",
-            "eta_decode_screened_ragged", "eta_decode_dense_ragged")
+            "eta_decode_screened_ragged", "eta_decode_dense_ragged", "eta_build_block_meta_paged",
+            "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -252,6 +266,49 @@ def decode_dense_ragged(shape: Shape, params: Params, q, k, v, seq_lens: torch.T
     _check(lib.eta_decode_dense_ragged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
                                        _ptr(seq_lens), max_tokens, _ptr(tau), tau_batch_stride, _ptr(out),
                                        _ptr(ws), ws.numel(), _stream(stream)), "eta_decode_dense_ragged")
+
+
+def _pages(block_table: torch.Tensor, num_pages: int) -> Pages:
+    return Pages(block_table.data_ptr(), num_pages)
+
+
+def build_block_meta_paged(shape: Shape, k_pool: torch.Tensor, block_table: torch.Tensor, num_pages: int,
+                           blk_begin: int, blk_end: int, mu, var, maxnorm, stream=None) -> None:
+    _check(lib.eta_build_block_meta_paged(ctypes.byref(shape), _ptr(k_pool), _pages(block_table, num_pages),
+                                          blk_begin, blk_end, Meta(mu.data_ptr(), var.data_ptr(), maxnorm.data_ptr()),
+                                          _stream(stream)), "eta_build_block_meta_paged")
+
+
+def decode_sparse_paged(shape: Shape, params: Params, q, k_pool, v_pool, block_table: torch.Tensor, num_pages: int,
+                        meta, seq_lens: torch.Tensor, max_tokens: int, out: torch.Tensor, ws: torch.Tensor,
+                        tau: Optional[torch.Tensor] = None, tau_batch_stride: int = 0, W=None, bias=None,
+                        tau_out=None, stream=None, **outs) -> None:
+    so = _screen_out(**outs)
+    t, w_, b_, to = _thr(tau, W, bias, tau_out)
+    _check(lib.eta_decode_sparse_paged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_pool),
+                                       _ptr(v_pool), _pages(block_table, num_pages),
+                                       Meta(*(m.data_ptr() for m in meta)), _ptr(seq_lens), max_tokens, t,
+                                       tau_batch_stride, w_, b_, to, _ptr(out),
+                                       ctypes.byref(so) if so is not None else None, _ptr(ws), ws.numel(),
+                                       _stream(stream)), "eta_decode_sparse_paged")
+
+
+def decode_screened_paged(shape: Shape, params: Params, q, k_pool, v_pool, block_table: torch.Tensor,
+                          num_pages: int, seq_lens: torch.Tensor, max_tokens: int, tau: torch.Tensor,
+                          tau_batch_stride: int, out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check(lib.eta_decode_screened_paged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_pool),
+                                         _ptr(v_pool), _pages(block_table, num_pages), _ptr(seq_lens), max_tokens,
+                                         _ptr(tau), tau_batch_stride, _ptr(out), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "eta_decode_screened_paged")
+
+
+def decode_dense_paged(shape: Shape, params: Params, q, k_pool, v_pool, block_table: torch.Tensor, num_pages: int,
+                       seq_lens: torch.Tensor, max_tokens: int, tau: Optional[torch.Tensor], tau_batch_stride: int,
+                       out: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    _check(lib.eta_decode_dense_paged(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k_pool),
+                                      _ptr(v_pool), _pages(block_table, num_pages), _ptr(seq_lens), max_tokens,
+                                      _ptr(tau), tau_batch_stride, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "eta_decode_dense_paged")
 
 
 def decode_sparse(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, tau: torch.Tensor,

@@ -121,21 +121,28 @@ eta_status_t check_params(const eta_params_t* p) {
 // Shapes the decode kernel can stage (two stages of a K and a V block plus its
 // fixed shared memory) and index (prefix table and partial counters of B*Hkv
 // entries).
-eta_status_t check_decode_shape(const eta_shape_t* s, bool dense) {
+eta_status_t check_decode_shape(const eta_shape_t* s, bool dense, int64_t pool_pages = 0) {
   (void)dense;  // both passes keep the same segment table
   const int BH = s->batch * s->n_kv_heads;
   if (BH > kMaxBH) return ETA_ERR_UNSUPPORTED;
   const int G = s->n_q_heads / s->n_kv_heads;
   const size_t tile = static_cast<size_t>(s->block_size) * s->head_dim * elem_bytes(s->kv_dtype);
-  const size_t fixed = static_cast<size_t>(8) * G * (s->head_dim + 2) * 4 + 16 +
+  const size_t fixed = static_cast<size_t>(8) * G * (s->head_dim + 2) * 4 + 16 + 64 +
                        static_cast<size_t>(BH + 1) * 4 + 64;
   const size_t need = 2 * (2 * tile + 32) + fixed;
   if (need + 1024 > static_cast<size_t>(device_max_smem_optin())) return ETA_ERR_UNSUPPORTED;
   // bf16 K/V with bf16 q take the tensor-core kernel, whose TMA tensor copies
   // address cache rows with 32-bit coordinates
-  if (s->kv_dtype == ETA_BF16 && s->q_dtype == ETA_BF16 &&
-      static_cast<int64_t>(BH) * s->capacity > static_cast<int64_t>(INT32_MAX))
-    return ETA_ERR_UNSUPPORTED;
+  const int64_t store_rows = pool_pages > 0 ? pool_pages * s->n_kv_heads * s->block_size
+                                           : static_cast<int64_t>(BH) * s->capacity;
+  // the kernels address store rows with 32-bit integers (TMA coordinates too)
+  if (store_rows > static_cast<int64_t>(INT32_MAX)) return ETA_ERR_UNSUPPORTED;
+  return ETA_OK;
+}
+
+// A paged pool: a block table and at least one page.
+eta_status_t check_pages(const eta_pages_t& pg) {
+  if (pg.block_table == nullptr || !aligned(pg.block_table, 4) || pg.num_pages < 1) return ETA_ERR_INVALID_ARG;
   return ETA_OK;
 }
 
@@ -212,8 +219,11 @@ eta_status_t check_common_decode(const eta_shape_t* s, const eta_params_t* p, co
 
 eta_status_t do_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k, const void* v,
                        int64_t n, const float* tau, int64_t tau_stride, float* out, const Workspace& w,
-                       cudaStream_t st, bool dense, const int32_t* seq_lens = nullptr) {
+                       cudaStream_t st, bool dense, const int32_t* seq_lens = nullptr,
+                       const eta_pages_t* pages = nullptr) {
   DecodeCall c;
+  c.block_table = pages ? pages->block_table : nullptr;
+  c.num_pages = pages ? pages->num_pages : 0;
   c.shape = *s;
   c.beta = p->beta;
   c.gate = p->gate;
@@ -484,6 +494,76 @@ ETA_API eta_status_t eta_read_device_status(const void* workspace, eta_stream_t 
   if (e != cudaSuccess) return ETA_ERR_CUDA;
   *status = static_cast<eta_status_t>(v);
   return ETA_OK;
+}
+
+ETA_API eta_status_t eta_build_block_meta_paged(const eta_shape_t* shape, const void* k_pool, eta_pages_t pages,
+                                                int64_t blk_begin, int64_t blk_end, eta_meta_t meta,
+                                                eta_stream_t stream) {
+  ETA_TRY(check_shape(shape));
+  ETA_TRY(check_meta(meta));
+  ETA_TRY(check_pages(pages));
+  if (k_pool == nullptr || !aligned(k_pool, 16)) return ETA_ERR_INVALID_ARG;
+  const int64_t nb_cap = shape->capacity / shape->block_size;
+  if (blk_begin < 0 || blk_end > nb_cap || blk_begin > blk_end) return ETA_ERR_INVALID_ARG;
+  if (blk_begin == blk_end) return ETA_OK;
+  return from_cuda(
+      launch_build_meta(*shape, k_pool, blk_begin, blk_end, meta, stream, pages.block_table, pages.num_pages));
+}
+
+ETA_API eta_status_t eta_decode_sparse_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                             const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                             eta_meta_t meta, const int32_t* seq_lens, int64_t max_tokens,
+                                             const float* tau, int64_t tau_batch_stride, const float* W,
+                                             const float* bias, float* tau_out, float* out,
+                                             const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
+                                             eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k_pool, v_pool, max_tokens, out));
+  ETA_TRY(check_pages(pages));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_screen_shape(shape));
+  ETA_TRY(check_decode_shape(shape, false, pages.num_pages));
+  ETA_TRY(check_meta(meta));
+  ETA_TRY(check_thresholds(shape, q, tau, tau_batch_stride, W, bias, tau_out));
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  const Workspace w = ws_carve(workspace, L);
+  const float* t = W ? tau_out : tau;
+  const int64_t ts = W ? shape->n_q_heads : tau_batch_stride;
+  ETA_TRY(do_screen(shape, params, q, meta, max_tokens, W ? nullptr : tau, W ? 0 : tau_batch_stride, extra, w,
+                    stream, W, bias, tau_out, seq_lens));
+  return do_decode(shape, params, q, k_pool, v_pool, max_tokens, t, ts, out, w, stream, false, seq_lens, &pages);
+}
+
+ETA_API eta_status_t eta_decode_screened_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                               const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                               const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                               int64_t tau_batch_stride, float* out, void* workspace,
+                                               size_t ws_bytes, eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k_pool, v_pool, max_tokens, out));
+  ETA_TRY(check_pages(pages));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_decode_shape(shape, false, pages.num_pages));
+  if (tau == nullptr || tau_batch_stride < 0 || !aligned(tau, 4)) return ETA_ERR_INVALID_ARG;
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_decode(shape, params, q, k_pool, v_pool, max_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L),
+                   stream, false, seq_lens, &pages);
+}
+
+ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                            const void* k_pool, const void* v_pool, eta_pages_t pages,
+                                            const int32_t* seq_lens, int64_t max_tokens, const float* tau,
+                                            int64_t tau_batch_stride, float* out, void* workspace, size_t ws_bytes,
+                                            eta_stream_t stream) {
+  ETA_TRY(check_common_decode(shape, params, q, k_pool, v_pool, max_tokens, out));
+  ETA_TRY(check_pages(pages));
+  ETA_TRY(check_lens(seq_lens));
+  ETA_TRY(check_decode_shape(shape, true, pages.num_pages));
+  if (tau != nullptr && (tau_batch_stride < 0 || !aligned(tau, 4))) return ETA_ERR_INVALID_ARG;
+  WsLayout L;
+  ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
+  return do_decode(shape, params, q, k_pool, v_pool, max_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L),
+                   stream, true, seq_lens, &pages);
 }
 
 }  // extern "C"

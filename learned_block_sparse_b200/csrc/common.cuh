@@ -135,6 +135,26 @@ __device__ __forceinline__ int64_t seq_len_of(const int32_t* seq_lens, int b, in
   return v;
 }
 
+// Where the keys (or values) of a logical block live. Contiguous caches are
+// [B][Hkv][capacity][d]; paged pools are [num_pages][Hkv][bs][d], row b's
+// logical block j in page block_table[b * max_blocks + j].
+struct KvLayout {
+  const int32_t* block_table;  // null: contiguous
+  int max_blocks, num_pages, Hkv, bs;
+  int64_t cap;
+};
+
+// Row, in a [rows][d] view of the store, of token 0 of logical block blk of
+// segment seg = b * Hkv + kvh; -1 when the page index is outside the pool.
+// (The host keeps every row index of a store below 2^31.)
+__device__ __forceinline__ int kv_block_row(const KvLayout& L, int seg, int blk) {
+  if (L.block_table == nullptr) return static_cast<int>(static_cast<int64_t>(seg) * L.cap + static_cast<int64_t>(blk) * L.bs);
+  const int b = seg / L.Hkv, kvh = seg - b * L.Hkv;
+  const int page = __ldg(L.block_table + static_cast<int64_t>(b) * L.max_blocks + blk);
+  if (page < 0 || page >= L.num_pages) return -1;
+  return (page * L.Hkv + kvh) * L.bs;
+}
+
 // Programmatic dependent launch. The screening and decode kernels are launched
 // with cudaLaunchAttributeProgrammaticStreamSerialization, so each may start
 // (launch, shared-memory and barrier set-up) while the kernel before it on the

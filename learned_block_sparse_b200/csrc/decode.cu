@@ -97,10 +97,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
     const uint64_t pol = l2_policy_evict_first();
     const KV* kb = static_cast<const KV*>(a.k);
     const KV* vb = static_cast<const KV*>(a.v);
-    auto issue = [&](int st, int seg, int blk, int rows) {
+    auto issue = [&](int st, int row0, int rows) {
       const uint32_t bytes = static_cast<uint32_t>(rows) * D * EB;
       mbar_arrive_expect_tx(&s_full[st], 2 * bytes);
-      const int64_t off = (static_cast<int64_t>(seg) * a.cap + static_cast<int64_t>(blk) * a.bs) * D;
+      const int64_t off = static_cast<int64_t>(row0) * D;
       bulk_g2s(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes, kb + off, bytes, &s_full[st], pol);
       bulk_g2s(s_tiles + (static_cast<size_t>(st) * 2 + 1) * tile_bytes, vb + off, bytes, &s_full[st], pol);
     };

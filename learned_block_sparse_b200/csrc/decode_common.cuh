@@ -20,6 +20,7 @@ struct DecodeArgs {
   const uint32_t* union_list;
   const int32_t* union_cnt;
   const int32_t* seq_lens;  // [B] per-row token counts, or null (every row has n)
+  KvLayout kv;              // contiguous cache or paged pool
   float* o_part;
   float2* ml_part;
   float* out;
@@ -173,7 +174,8 @@ __device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int
 // less when the ring has fewer stages, so PL consecutive positions never share
 // a stage and are armed in parallel): wait until the position's stage is free,
 // publish (block, head mask, rows, segment) in s_info and call
-// issue(stage, segment, block, rows), which must arm s_full[stage] (arrive +
+// issue(stage, row0, rows) (row0: the block's first row in the [rows][d] view
+// of the K and V stores), which must arm s_full[stage] (arrive +
 // expected bytes) and start the copies. The warp reads the union list 32
 // entries at a time, one batch ahead. A stage's r-th reuse waits for the
 // consumer release that completed the empty barrier's phase r-1.
@@ -185,34 +187,49 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
   int PL = kMaxPL;  // issuing lanes
   while (PL > NST) PL >>= 1;
   const int lane = threadIdx.x & 31;
-  // entry of position p: segment, (block << 8 | head mask) and the block's
-  // rows (tokens of the row inside the block; -1 when the block is past it)
-  auto load_entry = [&](int64_t p, int& seg, uint32_t& e, int& rows) {
+  // entry of position p, in two halves so the list load of the next batch is
+  // in flight while this batch is issued: fetch() gives the segment and
+  // (block << 8 | head mask); finish() the block's rows (tokens of the row
+  // inside it; -1 when the block is past the row or its page outside the pool)
+  // and the store row of its token 0
+  auto fetch = [&](int64_t p, int& seg, uint32_t& e) {
     seg = 0;
     e = 0;
-    rows = 0;
     if (p < hi) {
       seg = seg_of(p);
       const int64_t j = p - pre(seg);
       e = DENSE ? ((static_cast<uint32_t>(j) << 8) | ((1u << G) - 1u))
                 : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + j);
-      const int64_t r = seg_tokens(a, seg) - static_cast<int64_t>(e >> 8) * a.bs;
-      rows = r <= 0 ? -1 : (r < a.bs ? static_cast<int>(r) : a.bs);
     }
   };
-  int seg_cur, seg_nxt = 0, rows_cur, rows_nxt = 0;
+  auto finish = [&](int64_t p, int seg, uint32_t e, int& rows, int& row0) {
+    rows = 0;
+    row0 = 0;
+    if (p < hi) {
+      const int blk = static_cast<int>(e >> 8);
+      const int64_t r = seg_tokens(a, seg) - static_cast<int64_t>(blk) * a.bs;
+      rows = r <= 0 ? -1 : (r < a.bs ? static_cast<int>(r) : a.bs);
+      if (rows > 0) {
+        row0 = kv_block_row(a.kv, seg, blk);
+        if (row0 < 0) rows = -1;
+      }
+    }
+  };
+  int seg_cur, seg_nxt = 0, rows_cur, row_cur;
   uint32_t e_cur, e_nxt = 0;
-  load_entry(lo + lane, seg_cur, e_cur, rows_cur);
+  fetch(lo + lane, seg_cur, e_cur);
   int issued = 0;    // this lane: 1 + the last position (relative to lo) it armed
   int aborted = 0;
   for (int64_t base = lo; base < hi && !aborted; base += 32) {
-    if (base + 32 < hi) load_entry(base + 32 + lane, seg_nxt, e_nxt, rows_nxt);
+    finish(base + lane, seg_cur, e_cur, rows_cur, row_cur);
+    if (base + 32 < hi) fetch(base + 32 + lane, seg_nxt, e_nxt);
     const int cnt = static_cast<int>(hi - base < 32 ? hi - base : int64_t{32});
     for (int s = 0; s < cnt && !aborted; s += PL) {
       const int src = s + (lane < PL ? lane : 0);
       const int seg_i = __shfl_sync(kFull, seg_cur, src);
       const uint32_t e_i = __shfl_sync(kFull, e_cur, src);
       const int rows_i = __shfl_sync(kFull, rows_cur, src);
+      const int row_i = __shfl_sync(kFull, row_cur, src);
       if (lane < PL && src < cnt) {
         const int it = static_cast<int>(base - lo) + src;
         const int st = it % NST;
@@ -221,13 +238,13 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
         if (!aborted) {
           const int blk = static_cast<int>(e_i >> 8);
           int rows = rows_i;
-          if (rows < 0) {  // a list entry past the row's last block: load nothing
+          if (rows < 0) {  // a list entry past the row's last block, or a bad page: load nothing
             atomicExch(a.status, static_cast<int32_t>(ETA_ERR_INVALID_ARG));
             rows = 0;
           }
           s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
           if (rows == 0) mbar_arrive(&s_full[st]);
-          else issue(st, seg_i, blk, rows);
+          else issue(st, row_i, rows);
           issued = it + 1;
         }
       }
@@ -235,7 +252,6 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
     }
     seg_cur = seg_nxt;
     e_cur = e_nxt;
-    rows_cur = rows_nxt;
   }
   if (aborted && lane < PL) {
     // let the copies this lane armed land before the thread block can exit
@@ -265,6 +281,12 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.cap = s.capacity;
   a.n = c.n;
   a.seq_lens = c.seq_lens;
+  a.kv.block_table = c.block_table;
+  a.kv.max_blocks = static_cast<int>(s.capacity / s.block_size);
+  a.kv.num_pages = c.num_pages;
+  a.kv.Hkv = s.n_kv_heads;
+  a.kv.bs = s.block_size;
+  a.kv.cap = s.capacity;
   a.tau_stride = c.tau_stride;
   a.B = s.batch;
   a.Hq = s.n_q_heads;

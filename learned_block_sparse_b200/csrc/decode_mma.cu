@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   unsigned char* s_tiles = smem;
   uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * tile_bytes);
   uint64_t* s_empty = s_full + NST;
-  int4* s_info = reinterpret_cast<int4*>(s_empty + NST);
+  uint64_t* s_aux = s_empty + NST;  // [8] per issuing lane: copies of a partial block
+  int4* s_info = reinterpret_cast<int4*>(s_aux + 8);
   float* s_macc = reinterpret_cast<float*>(s_info + NST);  // [kMW][G][D]
   float* s_mm = s_macc + kMW * G * D;                      // [kMW][G]
   float* s_ml = s_mm + kMW * G;                            // [kMW][G]
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
     }
+    for (int s = 0; s < 8; ++s) mbar_init(&s_aux[s], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -171,18 +173,37 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   if (warp == kMW) {
     // ------------------------------------------------------------ producer
     const uint64_t pol = l2_policy_evict_first();
-    auto issue = [&](int st, int seg, int blk, int /*rows*/) {
-      // whole boxes land even for the partial last block (rows past the
-      // cache end read as zeros, rows past n are masked by the consumer)
-      mbar_arrive_expect_tx(&s_full[st], 2 * tile_bytes);
-      const int y = static_cast<int>(static_cast<int64_t>(seg) * a.cap + static_cast<int64_t>(blk) * bs);
+    uint32_t aux_phase = 0;  // this lane's partial-block barrier
+    auto issue = [&](int st, int row0, int rows) {
+      // whole boxes land even for a partial block (rows past the store's end
+      // read as zeros)
+      const int y = row0;
       unsigned char* kt = s_tiles + static_cast<size_t>(st) * 2 * tile_bytes;
       unsigned char* vt = kt + tile_bytes;
+      uint64_t* bar = rows == bs ? &s_full[st] : &s_aux[lane];
+      mbar_arrive_expect_tx(bar, 2 * tile_bytes);
 #pragma unroll
       for (int h = 0; h < D / 64; ++h) {
-        tma_load_2d(kt + h * bs * 128, &tmk, h * 64, y, &s_full[st], pol);
-        tma_load_2d(vt + h * bs * 128, &tmv, h * 64, y, &s_full[st], pol);
+        tma_load_2d(kt + h * bs * 128, &tmk, h * 64, y, bar, pol);
+        tma_load_2d(vt + h * bs * 128, &tmv, h * 64, y, bar, pol);
       }
+      if (rows == bs) return;
+      // Partial block: the store's rows past the row's last token may hold
+      // anything, NaN included. Their keys are masked by the consumer, but
+      // P = 0 times NaN would still reach O, so their values are zeroed here
+      // once the copies have landed, before the stage is handed over.
+      if (!mbar_wait_bounded(bar, aux_phase, s_abort, a.status)) {
+        const uint64_t t0 = global_timer_ns();  // copies still in flight: let them land
+        while (!mbar_try_wait(bar, aux_phase) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+      aux_phase ^= 1u;
+      for (int r = rows; r < bs; ++r)
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(vt + swz(bs, r, c)) = make_uint4(0u, 0u, 0u, 0u);
+      // generic-proxy writes: order them before the next TMA write into the stage
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&s_full[st]);
     };
     producer_loop<G, DENSE, kMW>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
     return;
@@ -424,7 +445,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const int BH = s.batch * s.n_kv_heads;
   const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
   constexpr int kMW = MmaWarps<D, CH>::kMW;
-  const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 +
+  const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 + 8 * sizeof(uint64_t) +
                        static_cast<size_t>(BH + 1) * sizeof(int32_t) + 1024;
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
   const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 512;
@@ -439,7 +460,8 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(nst) * per_stage + fixed + 64;
 
   CUtensorMap tmk, tmv;
-  const int64_t rows = static_cast<int64_t>(BH) * s.capacity;
+  const int64_t rows = c.block_table != nullptr ? static_cast<int64_t>(c.num_pages) * s.n_kv_heads * s.block_size
+                                                : static_cast<int64_t>(BH) * s.capacity;
   if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size))
     return cudaErrorInvalidValue;
 

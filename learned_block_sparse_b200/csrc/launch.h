@@ -72,7 +72,7 @@ cudaError_t launch_pdl(Kernel kernel, unsigned grid, unsigned block, size_t smem
 }
 
 cudaError_t launch_build_meta(const eta_shape_t& s, const void* k, int64_t b0, int64_t b1, const eta_meta_t& m,
-                              cudaStream_t st);
+                              cudaStream_t st, const int32_t* block_table = nullptr, int num_pages = 0);
 
 cudaError_t launch_predict(const eta_shape_t& s, const void* q, const float* W, const float* bias, float* tau,
                            cudaStream_t st);
@@ -104,6 +104,8 @@ struct DecodeCall {
   const void* v;
   int64_t n;               // tokens (all rows), or the upper bound of seq_lens
   const int32_t* seq_lens; // [B] per-row token counts (device), or null
+  const int32_t* block_table;  // [B][capacity/block_size] pages (device), or null: contiguous k, v
+  int num_pages;           // pages in the k and v pools (paged only)
   const float* tau;        // gate thresholds; null = -inf (dense only)
   int64_t tau_stride;
   float* out;

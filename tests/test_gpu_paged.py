@@ -1,0 +1,126 @@
+"""Paged KV pools (eta_*_paged): the K and V blocks of a contiguous cache are
+scattered into randomly permuted pages of a pool; metadata built from the pool
+and every decode result (lists, thresholds, outputs, dense outputs) must equal
+the contiguous per-row-length calls bit for bit (those are checked against the
+oracle in test_gpu_ragged.py). A page index outside the pool is reported in the
+device status word and never read."""
+import numpy as np
+import pytest
+import torch
+
+from learned_block_sparse_b200 import binding, synth
+from learned_block_sparse_b200.workload import DeviceWorkload
+
+pytestmark = pytest.mark.gpu
+
+
+def _pool(dw, seed, spare=7):
+    """Pools [pages][Hkv][bs][d] holding dw's K and V behind a permuted block table."""
+    w = dw.w
+    nbc = w.capacity // w.bs
+    pages = w.B * nbc + spare
+    g = torch.Generator().manual_seed(seed)
+    table = torch.randperm(pages, generator=g)[:w.B * nbc].view(w.B, nbc).to(torch.int32)
+    idx = table.view(-1).long().cuda()
+    pools = []
+    for src in (dw.K, dw.V):
+        blocks = src.view(w.B, w.Hkv, nbc, w.bs, w.d).permute(0, 2, 1, 3, 4).reshape(w.B * nbc, w.Hkv, w.bs, w.d)
+        pool = torch.full((pages, w.Hkv, w.bs, w.d), float("nan"), dtype=src.dtype, device="cuda")
+        pool[idx] = blocks
+        pools.append(pool)
+    return pools[0], pools[1], table.cuda(), pages
+
+
+def _lens(w, seed):
+    edge = [1, w.bs, w.bs + 1, w.n, 2 * w.bs - 1]
+    rng = np.random.default_rng(seed)
+    rest = list(rng.integers(1, w.n + 1, size=max(0, w.B - len(edge))))
+    return torch.tensor([int(x) for x in (edge + rest)[:w.B]], dtype=torch.int32, device="cuda")
+
+
+def _outs(w):
+    nb_cap = w.capacity // w.bs
+    return dict(active_idx=torch.full((w.B, w.Hq, nb_cap), -1, dtype=torch.int32, device="cuda"),
+                active_cnt=torch.zeros((w.B, w.Hq), dtype=torch.int32, device="cuda"),
+                union_list=torch.zeros((w.B, w.Hkv, nb_cap), dtype=torch.int32, device="cuda"),
+                union_cnt=torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda"))
+
+
+@pytest.mark.parametrize("dtype,Hq,Hkv,d,bs,mode", [
+    ("bf16", 8, 2, 128, 32, "predictor"),
+    ("bf16", 32, 4, 64, 64, "const"),
+    ("bf16", 4, 4, 128, 16, "const"),
+    ("f32", 4, 2, 64, 16, "predictor"),
+])
+def test_paged_pool_equals_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
+    w = synth.Workload("paged", dtype, 6, Hq, Hkv, d, bs * 50 + 3, bs, z=1.0, tau_mode=mode,
+                       densities=(0.3,), seed=700 + bs + Hq, offset_std=synth.SQRT_HALF)
+    dw = DeviceWorkload(w)
+    dec = dw.dec
+    k_pool, v_pool, table, pages = _pool(dw, seed=bs)
+    # metadata from the pool = metadata from the contiguous cache
+    mu = torch.full_like(dec.mu, float("nan"))
+    var = torch.full_like(dec.var, float("nan"))
+    mx = torch.full_like(dec.maxnorm, float("nan"))
+    nfull = w.n // w.bs
+    binding.build_block_meta_paged(dec.shape, k_pool, table, pages, 0, nfull, mu, var, mx)
+    torch.cuda.synchronize()
+    for a, b in ((mu, dec.mu), (var, dec.var)):
+        assert torch.equal(a[..., :nfull], b[..., :nfull])
+    assert torch.equal(mx[..., :nfull], dec.maxnorm[..., :nfull])
+
+    seq = _lens(w, seed=bs + 1)
+    if mode == "predictor":
+        calib = dw.calibrate(0.3)
+        thr = dict(W=dw.W, bias=calib[2])
+    else:
+        thr = dict(tau=dw.calibrate(0.3)[0], tau_batch_stride=0)
+    out_c = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    out_p = torch.empty_like(out_c)
+    tau_c = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
+    tau_p = torch.empty_like(tau_c)
+    oc, op = _outs(w), _outs(w)
+    extra_c = dict(tau_out=tau_c) if mode == "predictor" else {}
+    extra_p = dict(tau_out=tau_p) if mode == "predictor" else {}
+    binding.decode_sparse_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, seq, w.n, out_c, dec.ws,
+                                 **thr, **extra_c, **oc)
+    binding.decode_sparse_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, table, pages, (mu, var, mx), seq, w.n,
+                                out_p, dec.ws, **thr, **extra_p, **op)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for key in oc:
+        assert torch.equal(oc[key], op[key]), key
+    if mode == "predictor":
+        assert torch.equal(tau_c, tau_p)
+    assert torch.equal(out_c, out_p)
+    # the dense pass over the pool
+    dense_c = torch.empty_like(out_c)
+    dense_p = torch.empty_like(out_c)
+    binding.decode_dense_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, seq, w.n, None, 0, dense_c, dec.ws)
+    binding.decode_dense_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, table, pages, seq, w.n, None, 0,
+                               dense_p, dec.ws)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    assert torch.equal(dense_c, dense_p)
+
+
+def test_page_outside_the_pool_is_reported_and_not_read():
+    w = synth.WORKLOADS[3].replace(B=2, Hq=8, Hkv=2, n=32 * 30 + 5)
+    dw = DeviceWorkload(w)
+    dec = dw.dec
+    k_pool, v_pool, table, pages = _pool(dw, seed=3, spare=0)
+    seq = torch.tensor([w.n, w.n], dtype=torch.int32, device="cuda")
+    bad = table.clone()
+    bad[1, w.nb - 1] = pages          # the forced last block of row 1: always loaded
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    tau = torch.zeros((w.B, w.Hq), device="cuda")
+    binding.decode_sparse_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, bad, pages, dec.meta, seq, w.n, out,
+                                dec.ws, tau=tau, tau_batch_stride=w.Hq)
+    torch.cuda.synchronize()
+    assert dec.device_status() == binding.ETA_ERR_INVALID_ARG
+    good = torch.empty_like(out)
+    binding.decode_sparse_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, table, pages, dec.meta, seq, w.n,
+                                good, dec.ws, tau=tau, tau_batch_stride=w.Hq)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    assert torch.equal(out[0], good[0])   # row 0 does not touch the bad entry

@@ -169,3 +169,26 @@ def test_graph_replay_reads_the_new_lengths():
         assert torch.equal(replayed, direct), lens
     del g
     assert dw.dec.device_status() == 0
+
+
+@pytest.mark.parametrize("dtype,d,bs", [("bf16", 128, 32), ("bf16", 128, 16), ("bf16", 64, 64), ("f32", 64, 16)])
+def test_cache_rows_past_each_length_are_never_used(dtype, d, bs):
+    """Tokens at or past a row's length (the rest of its last block and beyond)
+    may hold anything: filling them with NaN changes no output bit."""
+    w = synth.Workload("tail", dtype, 5, 8, 2, d, bs * 40 + 9, bs, z=1.0, tau_mode="const",
+                       densities=(0.3,), seed=900 + bs + d, offset_std=synth.SQRT_HALF)
+    dw = DeviceWorkload(w)
+    tau = torch.zeros((w.Hq,), device="cuda")
+    lens = _lengths(w, seed=bs)
+    seq = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    a = dw.dec.step(dw.q, dw.K, dw.V, w.n, tau=tau, tau_batch_stride=0, seq_lens=seq).clone()
+    da = dw.dec.dense(dw.q, dw.K, dw.V, w.n, seq_lens=seq).clone()
+    for b, n_b in enumerate(lens):
+        dw.K[b, :, n_b:] = float("nan")
+        dw.V[b, :, n_b:] = float("nan")
+    b_ = dw.dec.step(dw.q, dw.K, dw.V, w.n, tau=tau, tau_batch_stride=0, seq_lens=seq).clone()
+    db = dw.dec.dense(dw.q, dw.K, dw.V, w.n, seq_lens=seq).clone()
+    torch.cuda.synchronize()
+    assert dw.dec.device_status() == 0
+    assert torch.isfinite(b_).all() and torch.isfinite(db).all()
+    assert torch.equal(a, b_) and torch.equal(da, db)
