@@ -62,8 +62,9 @@ def lib():
         L.oracle_screen_head.argtypes = [vp, i32, vp, vp, vp, i64, i32, f32, f32, f32, vp, vp]
         L.oracle_screen_head.restype = i32
         L.oracle_attend_head.argtypes = [i32, vp, vp, i32, i32, i64, vp, vp, i32, f32, f32, i32, vp]
+        L.oracle_block_stats.argtypes = [i32, vp, i32, i32, i64, i32, vp, f32, f32, f32, i32, vp, vp, vp]
         for fn in ("oracle_to_f32", "oracle_block_meta", "oracle_slice_meta",
-                   "oracle_predict_tau", "oracle_attend_head"):
+                   "oracle_predict_tau", "oracle_attend_head", "oracle_block_stats"):
             getattr(L, fn).restype = None
         _lib = L
     return _lib
@@ -201,6 +202,46 @@ def attend_head(k_slice, v_slice, bs: int, n: int, q_f32, blocks, tau: float,
     lib().oracle_attend_head(dt, _p(ka), _p(va), d, bs, n, _p(q_f32), _p(blocks),
                              int(blocks.size), float(tau), float(beta), int(gate), _p(out))
     return out
+
+
+def block_stats(k_slice, bs: int, n: int, q_f32, tau_screen: float, tau: float, beta: float,
+                gate: int = GATE_SIGMOID):
+    """Per block of one head's cache slice: (max scaled logit [nb] fp32, tokens
+    with S >= tau_screen [nb] int32, log-sum-exp of the gated logits [nb] f64)."""
+    ka, dt = _raw(k_slice)
+    q_f32 = np.ascontiguousarray(q_f32, np.float32)
+    d = q_f32.shape[0]
+    nb = (n + bs - 1) // bs
+    bmax = np.zeros((nb,), np.float32)
+    above = np.zeros((nb,), np.int32)
+    blse = np.zeros((nb,), np.float64)
+    lib().oracle_block_stats(dt, _p(ka), d, bs, n, nb, _p(q_f32), float(tau_screen), float(tau), float(beta),
+                             int(gate), _p(bmax), _p(above), _p(blse))
+    return bmax, above, blse
+
+
+def screen_diagnostics(bmax, above, blse, admitted, ns: int, tau_screen: float) -> dict:
+    """Table 16's screen quality for one head, over its ns screened blocks:
+    a block is truly active when its max logit reaches tau_screen;
+    false_negative = truly active blocks rejected / truly active blocks;
+    false_positive = admitted blocks not truly active / admitted blocks;
+    token_recall   = tokens with S >= tau_screen inside admitted blocks / all such tokens;
+    missed_mass    = dense gated softmax mass of the rejected blocks (all nb blocks
+                     in the normaliser)."""
+    adm = np.zeros((len(bmax),), bool)
+    adm[np.asarray(admitted, np.int64)] = True
+    scr = np.arange(len(bmax)) < ns
+    active = bmax >= np.float32(tau_screen)
+    a_s, adm_s = active & scr, adm & scr
+    lse_all = np.logaddexp.reduce(blse)
+    rejected = scr & ~adm
+    return {
+        "truly_active": int(a_s.sum()), "admitted": int(adm_s.sum()),
+        "false_negative": float((a_s & ~adm_s).sum() / max(1, a_s.sum())),
+        "false_positive": float((adm_s & ~a_s).sum() / max(1, adm_s.sum())),
+        "token_recall": float(above[scr & adm].sum() / max(1, above[scr].sum())),
+        "missed_mass": float(np.exp(np.logaddexp.reduce(blse[rejected]) - lse_all)) if rejected.any() else 0.0,
+    }
 
 
 def union_lists(lists_by_head, nb: int):

@@ -214,3 +214,54 @@ void oracle_attend_head(int kv_dtype, const void* k, const void* v, int d, int b
   free(g);
   free(pos);
 }
+
+/*
+ * Block statistics for the screen diagnostics of Table 16 (false negatives,
+ * false positives, token recall, missed mass), for one query head over the
+ * blocks [0, nb) of its cache slice, n tokens (t = n - 1 the current token):
+ *   S_s       = fl(fl(sum_i q_i k_si) * s), the sum by fused multiply-adds in
+ *               increasing i and s = fl(1/sqrt(d)) (fp32, so the comparisons
+ *               with the threshold below are reproducible bit for bit)
+ *   bmax[j]   = max over the block's tokens of S_s
+ *   above[j]  = number of the block's tokens with S_s >= tau_screen
+ *   blse[j]   = log sum over the block's tokens of exp(g_s), g_s the gated
+ *               logit of Eq. 2-3 (gate 0) or of strict mode (gate 1) with
+ *               threshold tau, the current token exempt (double)
+ * "Missed mass" of Table 16 is then sum over rejected j of exp(blse[j] - LSE)
+ * with LSE the log-sum-exp over all blocks: the fraction of the dense gated
+ * softmax mass that the screen dropped.
+ */
+void oracle_block_stats(int kv_dtype, const void* k, int d, int bs, int64_t n, int nb, const float* q,
+                        float tau_screen, float tau, float beta, int gate, float* bmax, int32_t* above,
+                        double* blse) {
+  const float s = (float)(1.0 / sqrt((double)d));
+  const int64_t t = n - 1;
+  for (int j = 0; j < nb; ++j) {
+    float mx = -INFINITY;
+    int cnt = 0;
+    double m = -INFINITY;
+    double gs_buf[1024];
+    int m_rows = 0;
+    for (int r = 0; r < bs; ++r) {
+      const int64_t tok = (int64_t)j * bs + r;
+      if (tok >= n) break;
+      float acc = 0.0f;
+      for (int i = 0; i < d; ++i) acc = fmaf(q[i], elem(k, kv_dtype, tok * d + i), acc);
+      const float S = acc * s;
+      if (S > mx) mx = S;
+      if (S >= tau_screen) ++cnt;
+      const double Sd = (double)S;
+      double g;
+      if (tok == t) g = Sd;
+      else if (gate == 0) g = Sd * sigmoid((double)beta * (Sd - (double)tau));
+      else g = (Sd >= (double)tau) ? Sd : -INFINITY;
+      gs_buf[m_rows++] = g;
+      if (g > m) m = g;
+    }
+    double z = 0.0;
+    for (int r = 0; r < m_rows; ++r) z += exp(gs_buf[r] - m);
+    bmax[j] = mx;
+    above[j] = cnt;
+    blse[j] = (m == -INFINITY) ? -INFINITY : m + log(z);
+  }
+}
