@@ -345,6 +345,27 @@ ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_
                                             eta_stream_t stream);
 
 /*
+ * eta_block_stats — the measurements behind the screen diagnostics of
+ * Table 16 (false negatives, false positives, token recall, missed mass). A
+ * dense pass over K (not a decode step): for every query head h and block
+ * j < ceil(n_tokens / block_size), with S_s = fl(fl(sum_i q_i k_si) * s) (fused
+ * multiply-adds in increasing i, s = fl(1/sqrt(d))):
+ *   block_max[b][h][j] = max over the block's tokens of S_s
+ *   above[b][h][j]     = tokens of the block with S_s >= tau - a
+ *   block_lse[b][h][j] = log sum over the block's tokens of exp(g_s), g_s the
+ *                        gated logit of params->gate with threshold tau (the
+ *                        current token exempt)
+ * Outputs are [B][Hq][capacity / block_size] fp32 / int32 / fp32; entries of
+ * blocks past n_tokens are left untouched. The maxima and counts are
+ * reproducible bit for bit; a block is "truly active" when its max reaches
+ * tau - a, and the fraction of gated softmax mass in the blocks a screen
+ * rejected is sum_rejected exp(lse_j) / sum_all exp(lse_j).
+ */
+ETA_API eta_status_t eta_block_stats(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                     const void* k, int64_t n_tokens, const float* tau, int64_t tau_batch_stride,
+                                     float* block_max, int32_t* above, float* block_lse, eta_stream_t stream);
+
+/*
  * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and
  * without any device allocation. The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory when they

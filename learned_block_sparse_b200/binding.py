@@ -101,6 +101,8 @@ def _load():
     L.eta_decode_screened_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense_paged.restype = st
     L.eta_decode_dense_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
+    L.eta_block_stats.restype = st
+    L.eta_block_stats.argtypes = [P(Shape), P(Params), vp, vp, i64, vp, i64, vp, vp, vp, vp]
     L.eta_decode_screened.restype = st
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
@@ -119,7 +121,7 @@ EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta
             "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static",
             "eta_screen_predict", "eta_decode_sparse_predict", "eta_screen_ragged", "eta_decode_sparse_ragged",
             "eta_decode_screened_ragged", "eta_decode_dense_ragged", "eta_build_block_meta_paged",
-            "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged")
+            "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged", "eta_block_stats")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -309,6 +311,13 @@ def decode_dense_paged(shape: Shape, params: Params, q, k_pool, v_pool, block_ta
                                       _ptr(v_pool), _pages(block_table, num_pages), _ptr(seq_lens), max_tokens,
                                       _ptr(tau), tau_batch_stride, _ptr(out), _ptr(ws), ws.numel(),
                                       _stream(stream)), "eta_decode_dense_paged")
+
+
+def block_stats(shape: Shape, params: Params, q, k, n_tokens: int, tau: torch.Tensor, tau_batch_stride: int,
+                block_max: torch.Tensor, above: torch.Tensor, block_lse: torch.Tensor, stream=None) -> None:
+    _check(lib.eta_block_stats(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k), n_tokens, _ptr(tau),
+                               tau_batch_stride, _ptr(block_max), _ptr(above), _ptr(block_lse), _stream(stream)),
+           "eta_block_stats")
 
 
 def decode_sparse(shape: Shape, params: Params, q, k, v, meta, n_tokens: int, tau: torch.Tensor,

@@ -566,4 +566,31 @@ ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_
                    stream, true, seq_lens, &pages);
 }
 
+ETA_API eta_status_t eta_block_stats(const eta_shape_t* shape, const eta_params_t* params, const void* q,
+                                     const void* k, int64_t n_tokens, const float* tau, int64_t tau_batch_stride,
+                                     float* block_max, int32_t* above, float* block_lse, eta_stream_t stream) {
+  ETA_TRY(check_shape(shape));
+  ETA_TRY(check_params(params));
+  ETA_TRY(check_tokens(shape, n_tokens));
+  if (q == nullptr || k == nullptr || tau == nullptr || tau_batch_stride < 0) return ETA_ERR_INVALID_ARG;
+  if (block_max == nullptr || above == nullptr || block_lse == nullptr) return ETA_ERR_INVALID_ARG;
+  if (!aligned(q, elem_bytes(shape->q_dtype)) || !aligned(k, 16) || !aligned(tau, 4) || !aligned(block_max, 4) ||
+      !aligned(above, 4) || !aligned(block_lse, 4))
+    return ETA_ERR_INVALID_ARG;
+  StatsCall c;
+  c.shape = *shape;
+  c.q = q;
+  c.k = k;
+  c.n = n_tokens;
+  c.tau = tau;
+  c.tau_stride = tau_batch_stride;
+  c.beta = params->beta;
+  c.offset_a = params->offset_a;
+  c.gate = params->gate;
+  c.bmax = block_max;
+  c.above = above;
+  c.blse = block_lse;
+  return from_cuda(launch_block_stats(c, stream));
+}
+
 }  // extern "C"

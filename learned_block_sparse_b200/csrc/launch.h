@@ -115,6 +115,21 @@ struct DecodeCall {
 };
 cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st);
 
+struct StatsCall {
+  eta_shape_t shape;
+  const void* q;
+  const void* k;
+  int64_t n;
+  const float* tau;
+  int64_t tau_stride;
+  float beta, offset_a;
+  int gate;
+  float* bmax;             // [B][Hq][nb_cap]
+  int32_t* above;          // [B][Hq][nb_cap]
+  float* blse;             // [B][Hq][nb_cap]
+};
+cudaError_t launch_block_stats(const StatsCall& c, cudaStream_t st);
+
 // Largest B*Hkv the decode kernel's on-chip prefix table holds.
 constexpr int kMaxBH = 8192;
 // The workspace starts with a fixed header, the part that must be zero before
