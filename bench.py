@@ -56,6 +56,7 @@ def parse_args():
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-sweep", action="store_true", help="skip the other densities of the configuration")
+    p.add_argument("--no-diagnostics", action="store_true", help="skip the screen-quality pass (Table 16 metrics)")
     p.add_argument("--l2-flush", default="write+read", choices=["write", "write+read"],
                    help="between steps: write 512 MiB, or write then read 512 MiB so the timed step "
                         "does not also pay for writing back the flush's dirty lines")
@@ -526,6 +527,8 @@ def run_eta(args):
             if "dense" in line:
                 sw[str(dens)]["speedup_vs_dense"] = line["dense"]["ms_per_step"] / sms
         line["sweep"] = sw
+    if not args.no_diagnostics:
+        line["screen_quality"] = screen_quality(w, dw, main["tau"])
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(w, args, dw)
     if rank == 0:
@@ -533,6 +536,19 @@ def run_eta(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def screen_quality(w, dw, thresholds):
+    """The pages' Table 16 screen diagnostics for this workload at the main
+    density (a dense pass over K, outside every timed region)."""
+    from learned_block_sparse_b200 import binding, diagnostics
+    tau, stride, bias = thresholds
+    dec = dw.dec
+    if bias is not None:
+        binding.predict_tau(dec.shape, dw.q, dw.W, bias, dec.tau)
+        tau, stride = dec.tau, w.Hq
+    r = diagnostics.screen_diagnostics(dec, dw.q, dw.K, w.n, tau, stride)
+    return {k: r[k] for k in ("false_negative", "false_positive", "token_recall", "missed_mass")}
 
 
 def cpu_baseline(w, args, dw):
