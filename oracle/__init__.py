@@ -29,7 +29,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-F32, BF16 = 0, 1
+F32, BF16, FP8 = 0, 1, 2
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11", "-fPIC", "-shared"]
 
 
@@ -71,13 +71,16 @@ def lib():
 
 
 def _raw(x):
-    """numpy view of the stored bits: float32 stays float32, bf16 becomes uint16."""
+    """numpy view of the stored bits: float32 stays float32, bf16 becomes uint16,
+    fp8 e4m3 becomes uint8."""
     try:
         import torch
         if isinstance(x, torch.Tensor):
             x = x.detach().cpu().contiguous()
             if x.dtype == torch.bfloat16:
                 return x.view(torch.int16).numpy().view(np.uint16), BF16
+            if x.dtype == torch.float8_e4m3fn:
+                return x.view(torch.uint8).numpy(), FP8
             if x.dtype == torch.float32:
                 return x.numpy(), F32
             raise TypeError(f"unsupported dtype {x.dtype}")
@@ -86,6 +89,8 @@ def _raw(x):
     x = np.ascontiguousarray(x)
     if x.dtype == np.uint16:
         return x, BF16
+    if x.dtype == np.uint8:
+        return x, FP8
     if x.dtype == np.float32:
         return x, F32
     raise TypeError(f"unsupported dtype {x.dtype}")

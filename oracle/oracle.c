@@ -27,9 +27,20 @@
 
 #define OR_F32 0
 #define OR_BF16 1
+#define OR_FP8 2   /* e4m3, "fn" variant: bias 7, no infinities, S.1111.111 = NaN */
+
+/* e4m3 byte -> value, from the format's definition: (-1)^s 2^(e-7) (1 + m/8)
+ * for e > 0, (-1)^s 2^-6 (m/8) for e = 0. */
+static float e4m3(uint8_t b) {
+  const int s = b >> 7, e = (b >> 3) & 15, m = b & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return (float)(s ? -v : v);
+}
 
 static float elem(const void* base, int dtype, int64_t i) {
   if (dtype == OR_F32) return ((const float*)base)[i];
+  if (dtype == OR_FP8) return e4m3(((const uint8_t*)base)[i]);
   uint32_t bits = (uint32_t)((const uint16_t*)base)[i] << 16;
   float f;
   memcpy(&f, &bits, 4);
