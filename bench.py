@@ -197,7 +197,7 @@ class ClockSampler:
 def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
     """Algorithmic bytes of one step from the admitted counts.
     union_cnt [B][Hkv]; the last block of each list is partial when n % b != 0."""
-    eb = 2 if w.dtype == "bf16" else 4
+    eb = {"f32": 4, "bf16": 2, "fp8": 1}[w.dtype]
     row = w.d * eb
     last_rows = w.n - (w.nb - 1) * w.bs
     blocks = int(union_cnt.sum())
@@ -485,7 +485,7 @@ def run_eta(args):
     line = {
         "metric": "sparse decode queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8": "fp8", "f32": "f32"}[w.dtype],
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller; see DESIGN.md input recipe)",
         "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
                    "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
@@ -496,7 +496,7 @@ def run_eta(args):
         "phases_ms": {("screen+predict" if w.tau_mode == "predictor" else "screen"): main["ms_screen"],
                       "decode": main["ms_decode"]},
         "roofline": {"bound": "hbm",
-                     "kernel": ("decode_mma_kernel" if w.dtype == "bf16" else "decode_kernel") + " (split merge fused)",
+                     "kernel": ("decode_kernel" if w.dtype == "f32" else "decode_mma_kernel") + " (split merge fused)",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind, "traffic": measured_traffic(w.name, bm["union_blocks"]),
                      "bytes_per_launch": bm["decode_kernel"]},

@@ -63,12 +63,17 @@ typedef enum {
   ETA_ERR_DEVICE_TIMEOUT = 5  /* a device-side wait exceeded its limit */
 } eta_status_t;
 
-typedef enum { ETA_F32 = 0, ETA_BF16 = 1 } eta_dtype_t;
+/* ETA_FP8_E4M3: one byte per element, 1 sign, 4 exponent (bias 7) and 3
+ * mantissa bits, no infinities (the "fn" variant: S.1111.111 is NaN, 448 the
+ * largest value). K and V only; every stored value widens exactly. */
+typedef enum { ETA_F32 = 0, ETA_BF16 = 1, ETA_FP8_E4M3 = 2 } eta_dtype_t;
 
 /* Problem shape. Supported: head_dim in {64, 128}; block_size in
  * {16, 32, 64, 128}; n_q_heads a multiple of n_kv_heads with group size
  * Hq/Hkv in {1, 2, 4, 8}; capacity a positive multiple of block_size;
- * capacity / block_size < 2^24; dtypes ETA_F32 or ETA_BF16. */
+ * capacity / block_size < 2^24; q_dtype ETA_F32 or ETA_BF16; kv_dtype
+ * ETA_F32, ETA_BF16 or ETA_FP8_E4M3 (the last with a bf16 q and head_dim 128;
+ * ETA_ERR_UNSUPPORTED otherwise). */
 typedef struct {
   int32_t batch;        /* B */
   int32_t n_q_heads;    /* Hq */

@@ -33,6 +33,7 @@ class Shape(ctypes.Structure):
                 ("kv_dtype", ctypes.c_int32), ("q_dtype", ctypes.c_int32)]
 
 
+ETA_FP8_E4M3 = 2
 GATE_SIGMOID, GATE_HARD = 0, 1   # Eq. 2-3 multiplicative gate; strict mode (hard masking)
 
 
@@ -139,6 +140,8 @@ def _dtype_code(t: torch.dtype) -> int:
         return ETA_F32
     if t == torch.bfloat16:
         return ETA_BF16
+    if t == torch.float8_e4m3fn:
+        return ETA_FP8_E4M3
     raise TypeError(f"unsupported dtype {t}")
 
 

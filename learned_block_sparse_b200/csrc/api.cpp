@@ -88,14 +88,16 @@ namespace {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int elem_bytes(int dtype) { return dtype == ETA_BF16 ? 2 : 4; }
+int elem_bytes(int dtype) { return dtype == ETA_FP8_E4M3 ? 1 : (dtype == ETA_BF16 ? 2 : 4); }
 
 eta_status_t check_shape(const eta_shape_t* s) {
   if (s == nullptr) return ETA_ERR_INVALID_ARG;
   if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1 || s->head_dim < 1 || s->block_size < 1)
     return ETA_ERR_INVALID_ARG;
-  if (s->kv_dtype != ETA_F32 && s->kv_dtype != ETA_BF16) return ETA_ERR_INVALID_ARG;
+  if (s->kv_dtype != ETA_F32 && s->kv_dtype != ETA_BF16 && s->kv_dtype != ETA_FP8_E4M3) return ETA_ERR_INVALID_ARG;
   if (s->q_dtype != ETA_F32 && s->q_dtype != ETA_BF16) return ETA_ERR_INVALID_ARG;
+  // fp8 K/V run on the tensor-core decode only: bf16 queries, d = 128
+  if (s->kv_dtype == ETA_FP8_E4M3 && (s->q_dtype != ETA_BF16 || s->head_dim != 128)) return ETA_ERR_UNSUPPORTED;
   if (s->n_q_heads % s->n_kv_heads != 0) return ETA_ERR_INVALID_ARG;
   if (s->capacity <= 0 || s->capacity % s->block_size != 0) return ETA_ERR_INVALID_ARG;
   if (s->head_dim != 64 && s->head_dim != 128) return ETA_ERR_UNSUPPORTED;

@@ -13,10 +13,21 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kFull = 0xffffffffu;
 
 struct Bf16Raw { uint16_t bits; };
+struct Fp8Raw { uint8_t bits; };
 
 template <typename T> struct KvTraits;
 template <> struct KvTraits<float> { static constexpr int kBytes = 4; static constexpr int kDtype = ETA_F32; };
 template <> struct KvTraits<Bf16Raw> { static constexpr int kBytes = 2; static constexpr int kDtype = ETA_BF16; };
+template <> struct KvTraits<Fp8Raw> { static constexpr int kBytes = 1; static constexpr int kDtype = ETA_FP8_E4M3; };
+
+// e4m3 byte -> fp32, exactly: (-1)^s 2^(e-7) (1 + m/8) for e > 0, (-1)^s m 2^-9
+// for e = 0; S.1111.111 is NaN.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  float v = e == 0u ? static_cast<float>(m) * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  if (e == 15u && m == 7u) v = __uint_as_float(0x7fc00000u);
+  return (b & 0x80u) ? -v : v;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -35,8 +46,9 @@ __device__ __forceinline__ void widen16<float>(const uint4& w, float* x) {
   x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
 }
 
-// One stored element of a q / K buffer in either dtype, widened to fp32.
+// One stored element of a q / K buffer in any supported dtype, widened to fp32.
 __device__ __forceinline__ float load_elem(const void* p, int dtype, int64_t i) {
+  if (dtype == ETA_FP8_E4M3) return e4m3_to_float(static_cast<const uint8_t*>(p)[i]);
   if (dtype == ETA_BF16) {
     uint32_t b = static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16;
     return __uint_as_float(b);

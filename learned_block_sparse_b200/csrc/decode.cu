@@ -319,7 +319,8 @@ cudaError_t launch_decode_kd(const DecodeCall& c, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st) {
-  if (c.shape.kv_dtype == ETA_BF16 && c.shape.q_dtype == ETA_BF16) return launch_decode_mma(c, st);
+  if (c.shape.kv_dtype == ETA_FP8_E4M3 || (c.shape.kv_dtype == ETA_BF16 && c.shape.q_dtype == ETA_BF16))
+    return launch_decode_mma(c, st);
   if (c.shape.kv_dtype == ETA_BF16)
     return c.dense ? launch_decode_kd<Bf16Raw, true>(c, st) : launch_decode_kd<Bf16Raw, false>(c, st);
   return c.dense ? launch_decode_kd<float, true>(c, st) : launch_decode_kd<float, false>(c, st);

@@ -24,6 +24,7 @@
 // V comes from ldmatrix.trans. In QK^T, rows of the tiles beyond G are zero.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -35,12 +36,13 @@ namespace eta {
 namespace {
 
 // Consumer warps: 4, or 8 where a block carries more consumer work per byte
-// than a 32-token block at d=128: 16-token blocks (half the bytes per block
-// for the same fixed cost) and d=64 (twice the keys, hence twice the gate and
-// softmax work, per byte); plus one producer warp.
-template <int D, int CH>
+// than a 32-token bf16 block at d=128: 16-token blocks (half the bytes per
+// block for the same fixed cost), d=64 (twice the keys, hence twice the gate
+// and softmax work, per byte) and fp8 K/V (half the bytes, plus the
+// conversions); plus one producer warp.
+template <int D, int CH, bool FP8>
 struct MmaWarps {
-  static constexpr int kMW = (CH == 16 || D == 64) ? 8 : 4;
+  static constexpr int kMW = (CH == 16 || D == 64 || FP8) ? 8 : 4;
   static constexpr int kThreads = (kMW + 1) * 32;
 };
 
@@ -111,17 +113,66 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// fp8 K/V. Two e4m3 bytes of w, picked by the byte permutation `sel` into bits
+// 8-15 and 24-31, become an f16x2 of the same values times 2^-8: the sign,
+// the 4 exponent bits and the 3 mantissa bits move into the f16 fields
+// unchanged, so the f16 exponent is the e4m3 one read with bias 15 instead of
+// 7. Exact for every finite e4m3 value, subnormals included; the 2^8 is put
+// back on the logits and the output.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
+  uint32_t t;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w), "r"(0u), "r"(sel));
+  return (t & 0x80008000u) | ((t >> 1) & 0x3f803f80u);
+}
+constexpr uint32_t kSelB01 = 0x1404u;  // bytes 0, 1
+constexpr uint32_t kSelB23 = 0x3424u;  // bytes 2, 3
+constexpr uint32_t kSelB02 = 0x2404u;  // bytes 0, 2
+constexpr uint32_t kSelB13 = 0x3414u;  // bytes 1, 3
+
+// As mma_rows8 / mma_16816 with f16 operands.
+__device__ __forceinline__ void mma_rows8_f16(float& d0, float& d1, uint32_t a_lo, uint32_t a_hi, uint32_t b0,
+                                              uint32_t b1) {
+  [[maybe_unused]] float z2, z3;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %10, %11};"
+      : "+f"(d0), "+f"(d1), "=f"(z2), "=f"(z3)
+      : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.0f), "f"(0.0f));
+}
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // HARD: the strict-mode gate (keys below tau removed) instead of Eq. 2-3.
-template <int D, int G, bool DENSE, int CH, bool HARD>
-__global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
+// FP8: e4m3 K/V (d = 128). A 16-byte shared chunk then holds 16 dims of one
+// key, so an ldmatrix fragment gives a thread dims 4q..4q+3 of one key (q =
+// lane % 4); the k slots of the f16 mma take them in that order (slots 2q,
+// 2q+1 <- dims 4q, 4q+1; slots 2q+8, 2q+9 <- dims 4q+2, 4q+3) and the query
+// fragments follow the same order, which leaves every dot product unchanged.
+// For P V the transposed fragment holds two keys x two dims; the byte
+// permutation splits it into the even-dim and the odd-dim n-tile.
+template <int D, int G, bool DENSE, int CH, bool HARD, bool FP8>
+__global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv) {
   constexpr int KST = D / 16;  // k-steps of QK^T
   constexpr int NDT = D / 8;   // n-tiles of PV
   static_assert(G >= 1 && G <= 8, "group size");
   static_assert(CH == 16 || CH == 32, "keys per chunk");
-  constexpr int kMW = MmaWarps<D, CH>::kMW;
-  constexpr int kMmaThreads = MmaWarps<D, CH>::kThreads;
+  constexpr int kMW = MmaWarps<D, CH, FP8>::kMW;
+  constexpr int kMmaThreads = MmaWarps<D, CH, FP8>::kThreads;
+  constexpr int EB = FP8 ? 1 : 2;  // bytes per element
+  static_assert(!FP8 || D == 128, "fp8 K/V: d = 128");
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   unsigned char* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -129,7 +180,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
   const int BH = a.B * a.Hkv;
   const int NST = a.nstages;
   const int bs = a.bs;
-  const uint32_t tile_bytes = static_cast<uint32_t>(bs) * D * 2;
+  const uint32_t tile_bytes = static_cast<uint32_t>(bs) * D * EB;
   unsigned char* s_tiles = smem;
   uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * tile_bytes);
   uint64_t* s_empty = s_full + NST;
@@ -182,10 +233,11 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
       unsigned char* vt = kt + tile_bytes;
       uint64_t* bar = rows == bs ? &s_full[st] : &s_aux[lane];
       mbar_arrive_expect_tx(bar, 2 * tile_bytes);
+      constexpr int kBoxElems = 128 / EB;  // a box row is 128 bytes
 #pragma unroll
-      for (int h = 0; h < D / 64; ++h) {
-        tma_load_2d(kt + h * bs * 128, &tmk, h * 64, y, bar, pol);
-        tma_load_2d(vt + h * bs * 128, &tmv, h * 64, y, bar, pol);
+      for (int h = 0; h < D / kBoxElems; ++h) {
+        tma_load_2d(kt + h * bs * 128, &tmk, h * kBoxElems, y, bar, pol);
+        tma_load_2d(vt + h * bs * 128, &tmv, h * kBoxElems, y, bar, pol);
       }
       if (rows == bs) return;
       // Partial block: the store's rows past the row's last token may hold
@@ -200,7 +252,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
       aux_phase ^= 1u;
       for (int r = rows; r < bs; ++r)
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) *reinterpret_cast<uint4*>(vt + swz(bs, r, c)) = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < D * EB / 16; ++c) *reinterpret_cast<uint4*>(vt + swz(bs, r, c)) = make_uint4(0u, 0u, 0u, 0u);
       // generic-proxy writes: order them before the next TMA write into the stage
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&s_full[st]);
@@ -225,9 +277,16 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
           static_cast<const uint16_t*>(a.q) + (static_cast<int64_t>(b) * a.Hq + kvh * G + row) * D;
 #pragma unroll
       for (int kk = 0; kk < KST; ++kk) {
-        const int c = 16 * kk + 2 * qd;
-        qa[kk][0] = static_cast<uint32_t>(qp[c]) | (static_cast<uint32_t>(qp[c + 1]) << 16);
-        qa[kk][1] = static_cast<uint32_t>(qp[c + 8]) | (static_cast<uint32_t>(qp[c + 9]) << 16);
+        if constexpr (FP8) {  // f16 fragments in the key fragments' dim order (see the kernel comment)
+          const int c = 16 * kk + 4 * qd;
+          auto f = [&](int i) { return __uint_as_float(static_cast<uint32_t>(qp[c + i]) << 16); };
+          qa[kk][0] = pack_f16x2(f(0), f(1));
+          qa[kk][1] = pack_f16x2(f(2), f(3));
+        } else {
+          const int c = 16 * kk + 2 * qd;
+          qa[kk][0] = static_cast<uint32_t>(qp[c]) | (static_cast<uint32_t>(qp[c + 1]) << 16);
+          qa[kk][1] = static_cast<uint32_t>(qp[c + 8]) | (static_cast<uint32_t>(qp[c + 9]) << 16);
+        }
       }
       tau_r = a.tau != nullptr ? a.tau[b * a.tau_stride + kvh * G + row] : -INFINITY;
     } else {
@@ -247,8 +306,14 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     if (live_row) {
 #pragma unroll
       for (int j = 0; j < NDT; ++j) {
-        s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0] + o[j][2];
-        s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1] + o[j][3];
+        if constexpr (FP8) {  // n-tile 2g + p holds dims 16g + 2c + p; values carry the 2^-8
+          const int base = 16 * (j >> 1) + (j & 1);
+          s_macc[(warp * G + row) * D + base + 4 * qd] = (o[j][0] + o[j][2]) * 256.0f;
+          s_macc[(warp * G + row) * D + base + 4 * qd + 2] = (o[j][1] + o[j][3]) * 256.0f;
+        } else {
+          s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0] + o[j][2];
+          s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1] + o[j][3];
+        }
       }
       if (qd == 0) {
         s_mm[warp * G + row] = m_r;
@@ -267,6 +332,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
     return Sv * rcp_approx(1.0f + ex2_approx(nbl * (Sv - tau_r))) * kLog2e;
   };
 
+  // fp8 keys enter the mma scaled by 2^-8 (exact): the logit scale takes it back
+  const float qscale = FP8 ? a.qscale * 256.0f : a.qscale;
   auto process = [&](int st, const int4 inf) {
     const uint32_t kt = smem_u32(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes);
     const uint32_t vt = kt + tile_bytes;
@@ -281,18 +348,40 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
       float se[NT][2], so[NT][2];
 #pragma unroll
       for (int j = 0; j < NT; ++j) se[j][0] = se[j][1] = so[j][0] = so[j][1] = 0.0f;
+      if constexpr (FP8) {
+        // a 16-byte chunk is one k-step: an x4 load gives 4 k-steps of one n-tile
 #pragma unroll
-      for (int k2 = 0; k2 < KST / 2; ++k2) {
-        uint32_t bb[NT][4];
+        for (int k4 = 0; k4 < KST / 4; ++k4) {
+          uint32_t bb[NT][4];
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-          ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k2 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
-                  bb[j][3]);
+          for (int j = 0; j < NT; ++j)
+            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k4 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+                    bb[j][3]);
 #pragma unroll
-        for (int j = 0; j < NT; ++j) mma_rows8(se[j][0], se[j][1], qa[2 * k2][0], qa[2 * k2][1], bb[j][0], bb[j][1]);
+          for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int j = 0; j < NT; ++j)
-          mma_rows8(so[j][0], so[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], bb[j][2], bb[j][3]);
+            for (int j = 0; j < NT; ++j) {
+              const uint32_t b0 = e4m3x2_to_f16x2_scaled(bb[j][m], kSelB01);
+              const uint32_t b1 = e4m3x2_to_f16x2_scaled(bb[j][m], kSelB23);
+              if (m & 1) mma_rows8_f16(so[j][0], so[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
+              else mma_rows8_f16(se[j][0], se[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
+            }
+        }
+      } else {
+#pragma unroll
+        for (int k2 = 0; k2 < KST / 2; ++k2) {
+          uint32_t bb[NT][4];
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k2 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+                    bb[j][3]);
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+            mma_rows8(se[j][0], se[j][1], qa[2 * k2][0], qa[2 * k2][1], bb[j][0], bb[j][1]);
+#pragma unroll
+          for (int j = 0; j < NT; ++j)
+            mma_rows8(so[j][0], so[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], bb[j][2], bb[j][3]);
+        }
       }
       // gate (Eq. 2-3) and online softmax on this thread's row
       float g[NT][2];
@@ -302,7 +391,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
         for (int j = 0; j < NT; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float v = row_on ? gate((se[j][e] + so[j][e]) * a.qscale) : -INFINITY;
+            const float v = row_on ? gate((se[j][e] + so[j][e]) * qscale) : -INFINITY;
             g[j][e] = v;
             bm = fmaxf(bm, v);
           }
@@ -314,7 +403,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
             const int key = c0 + 8 * j + 2 * qd + e;
             float v = -INFINITY;
             if (row_on && key < rows) {
-              const float Sv = (se[j][e] + so[j][e]) * a.qscale;
+              const float Sv = (se[j][e] + so[j][e]) * qscale;
               // the current token is exempt from the gate (Eq. 3)
               v = (tok0 + key == t_cur) ? Sv * kLog2e : gate(Sv);
             }
@@ -351,23 +440,46 @@ __global__ void __launch_bounds__(MmaWarps<D, CH>::kThreads, 1)
           o[j][3] *= corr;
         }
       }
-      // O += P V, P = high + low parts in bf16
+      // O += P V, P = high + low parts (bf16, or f16 with fp8 values)
 #pragma unroll
       for (int m2 = 0; m2 < NT / 2; ++m2) {
-        const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
-        const uint32_t h1 = pack_bf16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
-        const __nv_bfloat162 hb0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
-        const __nv_bfloat162 hb1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
-        const uint32_t l0 = pack_bf16x2(p[2 * m2][0] - __low2float(hb0), p[2 * m2][1] - __high2float(hb0));
-        const uint32_t l1 = pack_bf16x2(p[2 * m2 + 1][0] - __low2float(hb1), p[2 * m2 + 1][1] - __high2float(hb1));
         const int vrow = c0 + 16 * m2 + 8 * ((lane >> 3) & 1) + (lane & 7);
+        if constexpr (FP8) {
+          const uint32_t h0 = pack_f16x2(p[2 * m2][0], p[2 * m2][1]);
+          const uint32_t h1 = pack_f16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
+          const __half2 hh0 = *reinterpret_cast<const __half2*>(&h0);
+          const __half2 hh1 = *reinterpret_cast<const __half2*>(&h1);
+          const uint32_t l0 = pack_f16x2(p[2 * m2][0] - __low2float(hh0), p[2 * m2][1] - __high2float(hh0));
+          const uint32_t l1 = pack_f16x2(p[2 * m2 + 1][0] - __low2float(hh1), p[2 * m2 + 1][1] - __high2float(hh1));
+          // one x4 transposed load: keys 0-7 / 8-15 of dim chunks g and g+1 (16 dims each)
 #pragma unroll
-        for (int jd = 0; jd < NDT; jd += 2) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
-          // A rows 0-7: high part, rows 8-15: low part of the same P row
-          mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
-          mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
+          for (int g = 0; g < D / 16; g += 2) {
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_t(vt + swz(bs, vrow, g + (lane >> 4)), r0, r1, r2, r3);
+            mma_16816_f16(o[2 * g], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r0, kSelB02),
+                          e4m3x2_to_f16x2_scaled(r1, kSelB02));
+            mma_16816_f16(o[2 * g + 1], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r0, kSelB13),
+                          e4m3x2_to_f16x2_scaled(r1, kSelB13));
+            mma_16816_f16(o[2 * g + 2], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r2, kSelB02),
+                          e4m3x2_to_f16x2_scaled(r3, kSelB02));
+            mma_16816_f16(o[2 * g + 3], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r2, kSelB13),
+                          e4m3x2_to_f16x2_scaled(r3, kSelB13));
+          }
+        } else {
+          const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
+          const uint32_t h1 = pack_bf16x2(p[2 * m2 + 1][0], p[2 * m2 + 1][1]);
+          const __nv_bfloat162 hb0 = *reinterpret_cast<const __nv_bfloat162*>(&h0);
+          const __nv_bfloat162 hb1 = *reinterpret_cast<const __nv_bfloat162*>(&h1);
+          const uint32_t l0 = pack_bf16x2(p[2 * m2][0] - __low2float(hb0), p[2 * m2][1] - __high2float(hb0));
+          const uint32_t l1 = pack_bf16x2(p[2 * m2 + 1][0] - __low2float(hb1), p[2 * m2 + 1][1] - __high2float(hb1));
+#pragma unroll
+          for (int jd = 0; jd < NDT; jd += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
+            // A rows 0-7: high part, rows 8-15: low part of the same P row
+            mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
+            mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
+          }
         }
       }
     }
@@ -426,34 +538,37 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [rows][d] bf16 view of a K or V cache, boxes of [bs][64] with 128-byte swizzle.
-bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int bs) {
+// [rows][d] view of a K or V store (bf16, or fp8 bytes), boxes of [bs] rows of
+// 128 bytes with the 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int bs, bool fp8) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
+  const int eb = fp8 ? 1 : 2;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * eb};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(bs)};
   const cuuint32_t estride[2] = {1u, 1u};
-  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim, gstride, box, estride,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+             gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G, bool DENSE, int CH>
+template <int D, int G, bool DENSE, int CH, bool FP8>
 cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
-  const size_t tile = static_cast<size_t>(s.block_size) * D * 2;
-  constexpr int kMW = MmaWarps<D, CH>::kMW;
+  const size_t tile = static_cast<size_t>(s.block_size) * D * (FP8 ? 1 : 2);
+  constexpr int kMW = MmaWarps<D, CH, FP8>::kMW;
+  constexpr unsigned kThreads = MmaWarps<D, CH, FP8>::kThreads;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 + 8 * sizeof(uint64_t) +
                        static_cast<size_t>(BH + 1) * sizeof(int32_t) + 1024;
   const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
   const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 512;
   if (fixed + 2 * per_stage > budget) return cudaErrorInvalidValue;
-  // ~200 KB of stages: the consumer warps hold up to 4, the rest are in flight.
+  // ~200 KB of stages: the consumer warps hold up to kMW, the rest are in flight.
   const size_t nst_bw = (200 * 1024) / (2 * tile), nst_fit = (budget - fixed) / per_stage;
   int nst = static_cast<int>(nst_bw < nst_fit ? nst_bw : nst_fit);
-  nst = max(2, min(nst, 24));
+  nst = max(2, min(nst, FP8 ? 32 : 24));
   // With at least 2*kMW stages, round down to a multiple of kMW so a stage
   // always returns to the warp that released it (see the consumer loop).
   if (nst >= 2 * kMW) nst -= nst % kMW;
@@ -462,46 +577,55 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   CUtensorMap tmk, tmv;
   const int64_t rows = c.block_table != nullptr ? static_cast<int64_t>(c.num_pages) * s.n_kv_heads * s.block_size
                                                 : static_cast<int64_t>(BH) * s.capacity;
-  if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size))
+  if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size, FP8) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size, FP8))
     return cudaErrorInvalidValue;
 
   const DecodeArgs a = make_decode_args(c, nst);
   if (c.gate == ETA_GATE_HARD) {
     static std::atomic<uint64_t> smem_done{0};
-    cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, true>));
+    const void* fn = reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, true, FP8>);
+    cudaError_t e = allow_max_smem(smem_done, fn);
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, true>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads,
-                      smem, st, a, tmk, tmv);
+    return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, true, FP8>, static_cast<unsigned>(c.S), kThreads, smem, st,
+                      a, tmk, tmv);
   }
   static std::atomic<uint64_t> smem_done{0};
-  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, false>));
+  const void* fn = reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, false, FP8>);
+  cudaError_t e = allow_max_smem(smem_done, fn);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, false>, static_cast<unsigned>(c.S), MmaWarps<D, CH>::kThreads,
-                    smem, st, a, tmk, tmv);
+  return launch_pdl(decode_mma_kernel<D, G, DENSE, CH, false, FP8>, static_cast<unsigned>(c.S), kThreads, smem, st,
+                    a, tmk, tmv);
 }
 
-template <int D, bool DENSE, int CH>
+template <int D, bool DENSE, int CH, bool FP8>
 cudaError_t launch_mma_g(const DecodeCall& c, cudaStream_t st) {
   switch (c.shape.n_q_heads / c.shape.n_kv_heads) {
-    case 1: return launch_mma_t<D, 1, DENSE, CH>(c, st);
-    case 2: return launch_mma_t<D, 2, DENSE, CH>(c, st);
-    case 4: return launch_mma_t<D, 4, DENSE, CH>(c, st);
-    case 8: return launch_mma_t<D, 8, DENSE, CH>(c, st);
+    case 1: return launch_mma_t<D, 1, DENSE, CH, FP8>(c, st);
+    case 2: return launch_mma_t<D, 2, DENSE, CH, FP8>(c, st);
+    case 4: return launch_mma_t<D, 4, DENSE, CH, FP8>(c, st);
+    case 8: return launch_mma_t<D, 8, DENSE, CH, FP8>(c, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-// Chunks of 32 keys, or 16 for 16-token blocks.
-template <int D, bool DENSE>
+// Chunks of 32 keys, or 16 for 16-token blocks and for fp8 K/V (whose
+// conversions need the registers of the second half-chunk).
+template <int D, bool DENSE, bool FP8>
 cudaError_t launch_mma_c(const DecodeCall& c, cudaStream_t st) {
-  return c.shape.block_size == 16 ? launch_mma_g<D, DENSE, 16>(c, st) : launch_mma_g<D, DENSE, 32>(c, st);
+  if (FP8 || c.shape.block_size == 16) return launch_mma_g<D, DENSE, 16, FP8>(c, st);
+  return launch_mma_g<D, DENSE, (FP8 ? 16 : 32), FP8>(c, st);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_mma(const DecodeCall& c, cudaStream_t st) {
-  if (c.shape.head_dim == 128) return c.dense ? launch_mma_c<128, true>(c, st) : launch_mma_c<128, false>(c, st);
-  return c.dense ? launch_mma_c<64, true>(c, st) : launch_mma_c<64, false>(c, st);
+  if (c.shape.kv_dtype == ETA_FP8_E4M3) {
+    if (c.shape.head_dim != 128) return cudaErrorInvalidValue;
+    return c.dense ? launch_mma_c<128, true, true>(c, st) : launch_mma_c<128, false, true>(c, st);
+  }
+  if (c.shape.head_dim == 128)
+    return c.dense ? launch_mma_c<128, true, false>(c, st) : launch_mma_c<128, false, false>(c, st);
+  return c.dense ? launch_mma_c<64, true, false>(c, st) : launch_mma_c<64, false, false>(c, st);
 }
 
 }  // namespace eta

@@ -115,6 +115,7 @@ cudaError_t launch_meta_t(const eta_shape_t& s, const void* k, int64_t b0, int64
 
 cudaError_t launch_build_meta(const eta_shape_t& s, const void* k, int64_t b0, int64_t b1, const eta_meta_t& m,
                               cudaStream_t st, const int32_t* table, int num_pages) {
+  if (s.kv_dtype == ETA_FP8_E4M3) return launch_meta_t<Fp8Raw, 128>(s, k, b0, b1, m, st, table, num_pages);
   if (s.kv_dtype == ETA_BF16) {
     return s.head_dim == 128 ? launch_meta_t<Bf16Raw, 128>(s, k, b0, b1, m, st, table, num_pages)
                              : launch_meta_t<Bf16Raw, 64>(s, k, b0, b1, m, st, table, num_pages);

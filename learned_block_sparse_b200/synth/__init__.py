@@ -77,7 +77,7 @@ def normal_at(seed: int, stream: int, f: int) -> float:
 class Workload:
     """One decode-step workload. ``n`` counts cached tokens including the current one."""
     name: str
-    dtype: str           # storage dtype of q, K, V: "f32" or "bf16"
+    dtype: str           # storage dtype of K, V: "f32", "bf16" or "fp8" (e4m3; q then bf16)
     B: int
     Hq: int
     Hkv: int
@@ -117,10 +117,17 @@ class Workload:
 
     @property
     def dtype_code(self) -> int:
+        """Generator dtype of q (and of K, V before an fp8 rounding)."""
         return F32 if self.dtype == "f32" else BF16
 
     @property
     def torch_dtype(self):
+        """Storage dtype of K and V."""
+        return {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.float8_e4m3fn}[self.dtype]
+
+    @property
+    def q_torch_dtype(self):
+        """Storage dtype of q: bf16 with fp8 K/V."""
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
 
     def replace(self, **kw) -> "Workload":
@@ -132,7 +139,8 @@ SQRT_HALF = math.sqrt(0.5)
 # The decode configurations (names state the shapes). 1-5 are the parity and
 # benchmark workloads; 6 is the attention shape of the pages' block-size /
 # chunk-size table (Table 10: batch 64, 512K tokens, 32 query / 4 KV heads of
-# dimension 64, blocks of 64), calibrated to the union densities quoted there.
+# dimension 64, blocks of 64), calibrated to the union densities quoted there;
+# 7 is workload 3 with its K and V rounded to fp8 (e4m3).
 WORKLOADS = {
     1: Workload("tiny-f32-mha2-d64-n1024-b16", "f32", 1, 2, 2, 64, 1024, 16, z=1.5,
                 tau_mode="const", densities=(0.40,), seed=1001),
@@ -149,6 +157,9 @@ WORKLOADS = {
     6: Workload("gqa32x4-d64-n512k-b64-B64", "bf16", 64, 32, 4, 64, 524288, 64, z=1.0,
                 tau_mode="predictor", densities=(0.16, 0.355, 0.512), seed=1006,
                 offset_std=SQRT_HALF, density_kind="union"),
+    7: Workload("gqa32x8-d128-n128k-b32-B8-fp8", "fp8", 8, 32, 8, 128, 131072, 32, z=1.0,
+                tau_mode="predictor", densities=(0.20, 0.38, 0.60), seed=1003,
+                offset_std=SQRT_HALF),
 }
 WORKLOAD5_BATCHES = (1, 4, 16, 64)
 
@@ -163,7 +174,7 @@ def _empty(shape, dtype, pin: bool):
 def make_q(w: Workload, pin: bool = False) -> torch.Tensor:
     """q [B][Hq][d] ~ N(0,1) in the workload dtype."""
     lib = _load()
-    q = _empty((w.B, w.Hq, w.d), w.torch_dtype, pin)
+    q = _empty((w.B, w.Hq, w.d), w.q_torch_dtype, pin)
     lib.synth_normal_fill(w.seed, STREAM_Q, 0, q.numel(), 0.0, 1.0, w.dtype_code, q.data_ptr())
     return q
 
@@ -192,13 +203,18 @@ def fill_kv(w: Workload, q: torch.Tensor, which: str, dst: torch.Tensor, b0: int
     if is_k and needles is None:
         needles = make_needles(w)
     if w.capacity > w.n:
-        dst[:, :, w.n:, :].zero_()
-    lib.synth_fill_kv(w.seed, STREAM_K if is_k else STREAM_V, STREAM_OFFSET, w.dtype_code, w.B, w.Hkv,
-                      w.n, w.capacity, w.d, w.bs, b0, b1,
+        dst[:, :, w.n:, :].view(torch.uint8 if w.dtype == "fp8" else dst.dtype).zero_()
+    fp8 = w.dtype == "fp8"
+    # fp8 caches: drawn in fp32, then rounded to e4m3 (nearest even) by torch
+    out = torch.zeros(dst.shape, dtype=torch.float32) if fp8 else dst
+    lib.synth_fill_kv(w.seed, STREAM_K if is_k else STREAM_V, STREAM_OFFSET, F32 if fp8 else w.dtype_code, w.B,
+                      w.Hkv, w.n, w.capacity, w.d, w.bs, b0, b1,
                       w.offset_std if is_k else 0.0,
                       q.data_ptr(), w.dtype_code, w.Hq,
                       needles.data_ptr() if (is_k and needles is not None) else None,
-                      w.n_needles if is_k else 0, w.needle_scale, dst.data_ptr())
+                      w.n_needles if is_k else 0, w.needle_scale, out.data_ptr())
+    if fp8:
+        dst.copy_(out.to(torch.float8_e4m3fn))
     return dst
 
 

@@ -27,7 +27,7 @@ class DeviceWorkload:
         shp = (w.B, w.Hkv, w.capacity, w.d)
         self.K = torch.empty(shp, dtype=w.torch_dtype, device=self.device)
         self.V = torch.empty(shp, dtype=w.torch_dtype, device=self.device)
-        per_b = w.Hkv * w.capacity * w.d * (2 if w.dtype == "bf16" else 4)
+        per_b = w.Hkv * w.capacity * w.d * {"f32": 4, "bf16": 2, "fp8": 1}[w.dtype]
         bchunk = max(1, min(w.B, stage_bytes // max(1, per_b)))
         self.K_host = self.V_host = None
         if keep_host:
@@ -45,7 +45,7 @@ class DeviceWorkload:
                     torch.cuda.current_stream(self.device).synchronize()
             del stage
         self.dec = binding.EtaDecoder(w.B, w.Hq, w.Hkv, w.d, w.bs, w.capacity, kv_dtype=w.torch_dtype,
-                                      q_dtype=w.torch_dtype, beta=w.beta, z=w.z, offset_a=offset_a,
+                                      q_dtype=w.q_torch_dtype, beta=w.beta, z=w.z, offset_a=offset_a,
                                       n_local=w.n_local, n_splits=n_splits, device=self.device, gate=gate)
         self.dec.build_meta(self.K, 0, w.n // w.bs)
         self.W = self.bias0 = None

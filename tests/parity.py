@@ -17,7 +17,7 @@ import torch
 import oracle
 from learned_block_sparse_b200 import binding, synth
 
-TOL = {"bf16": 2e-3, "f32": 1e-5}
+TOL = {"bf16": 2e-3, "fp8": 2e-3, "f32": 1e-5}
 _POOL = cf.ThreadPoolExecutor(max_workers=max(1, min(32, os.cpu_count() or 1)))
 
 

@@ -24,10 +24,16 @@ def _pool(dw, seed, spare=7):
     idx = table.view(-1).long().cuda()
     pools = []
     for src in (dw.K, dw.V):
-        blocks = src.view(w.B, w.Hkv, nbc, w.bs, w.d).permute(0, 2, 1, 3, 4).reshape(w.B * nbc, w.Hkv, w.bs, w.d)
-        pool = torch.full((pages, w.Hkv, w.bs, w.d), float("nan"), dtype=src.dtype, device="cuda")
+        # scatter the raw bits (works for every storage dtype); unused pages hold NaN codes
+        raw = src.view(torch.uint8 if src.element_size() == 1 else
+                       (torch.int16 if src.element_size() == 2 else torch.int32))
+        blocks = raw.view(w.B, w.Hkv, nbc, w.bs, w.d).permute(0, 2, 1, 3, 4).reshape(w.B * nbc, w.Hkv, w.bs, w.d)
+        nan = torch.full((1,), float("nan"), dtype=torch.float32).to(src.dtype if src.element_size() > 1 else
+                                                                     torch.float32)
+        pool = torch.empty((pages, w.Hkv, w.bs, w.d), dtype=raw.dtype, device="cuda")
+        pool.fill_(0x7f if src.element_size() == 1 else int(nan.view(raw.dtype).item()))
         pool[idx] = blocks
-        pools.append(pool)
+        pools.append(pool.view(src.dtype))
     return pools[0], pools[1], table.cuda(), pages
 
 
@@ -51,6 +57,7 @@ def _outs(w):
     ("bf16", 32, 4, 64, 64, "const"),
     ("bf16", 4, 4, 128, 16, "const"),
     ("f32", 4, 2, 64, 16, "predictor"),
+    ("fp8", 8, 2, 128, 64, "const"),
 ])
 def test_paged_pool_equals_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
     w = synth.Workload("paged", dtype, 6, Hq, Hkv, d, bs * 50 + 3, bs, z=1.0, tau_mode=mode,

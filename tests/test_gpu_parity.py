@@ -46,6 +46,7 @@ def _full_check(w, density=None, n_splits=0, offset_a=0.0, heads=None, dense=Fal
 @pytest.mark.parametrize("dtype,d,bs,n,cap", [
     ("f32", 64, 16, 1024, None), ("bf16", 128, 32, 32 * 70 + 5, 32 * 80),
     ("bf16", 64, 64, 64 * 9, None), ("bf16", 128, 128, 128 * 5 + 100, None), ("f32", 128, 64, 64 * 7 + 1, None),
+    ("fp8", 128, 32, 32 * 33 + 7, None),
 ])
 def test_block_meta_bit_exact(dtype, d, bs, n, cap):
     w = synth.Workload("m", dtype, 2, 4, 2, d, n, bs, z=1.0, tau_mode="const", densities=(0.5,), seed=31,
@@ -126,7 +127,8 @@ def test_group_sizes(G):
 
 
 @pytest.mark.parametrize("dtype,d,bs", [("bf16", 64, 16), ("bf16", 64, 128), ("f32", 128, 32), ("f32", 64, 64),
-                                        ("bf16", 128, 128)])
+                                        ("bf16", 128, 128), ("fp8", 128, 16), ("fp8", 128, 32), ("fp8", 128, 64),
+                                        ("fp8", 128, 128)])
 def test_dtypes_dims_blocks(dtype, d, bs):
     w = synth.Workload("x", dtype, 2, 4, 2, d, bs * 37 + bs // 2 + 1, bs, z=1.0, tau_mode="const",
                        densities=(0.35,), seed=7 * d + bs, offset_std=synth.SQRT_HALF)
@@ -274,6 +276,16 @@ def test_strict_mode_gate(dtype, G, bs):
     heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
     orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, w.Hq, heads, gate=oracle.GATE_HARD)
     parity.compare(w, gpu, orc, heads)
+
+
+@pytest.mark.parametrize("G,density", [(1, 0.3), (4, 0.38), (8, 0.2)])
+def test_fp8_kv_workloads(G, density):
+    """fp8 (e4m3) K and V with bf16 queries, GQA groups up to 8, predictor
+    thresholds formed in the screen: lists bit-exact, outputs within 2e-3 of the
+    oracle reading the same fp8 bytes; the dense pass too."""
+    w = synth.Workload("fp8", "fp8", 2, 4 * G, 4, 128, 32 * 150 + 5, 32, z=1.0, tau_mode="predictor",
+                       densities=(density,), seed=600 + G, offset_std=synth.SQRT_HALF)
+    _full_check(w, density, dense=True)
 
 
 # ----------------------------------------------------------------- full size

@@ -81,6 +81,7 @@ def _compare(w, lens, outs, out, orc, check_lists=True):
     ("bf16", 32, 4, 64, 64, "const"),       # the pages' Table 10 head shape
     ("bf16", 4, 4, 128, 16, "const"),       # 16-token blocks, 8-warp decode
     ("f32", 4, 2, 64, 16, "predictor"),     # CUDA-core decode
+    ("fp8", 8, 2, 128, 32, "const"),        # fp8 K/V
 ])
 def test_ragged_rows_match_per_row_oracle(dtype, Hq, Hkv, d, bs, mode):
     w = synth.Workload("ragged", dtype, 7, Hq, Hkv, d, bs * 70 + 9, bs, z=1.0, tau_mode=mode,
@@ -171,7 +172,8 @@ def test_graph_replay_reads_the_new_lengths():
     assert dw.dec.device_status() == 0
 
 
-@pytest.mark.parametrize("dtype,d,bs", [("bf16", 128, 32), ("bf16", 128, 16), ("bf16", 64, 64), ("f32", 64, 16)])
+@pytest.mark.parametrize("dtype,d,bs", [("bf16", 128, 32), ("bf16", 128, 16), ("bf16", 64, 64), ("f32", 64, 16),
+                                        ("fp8", 128, 32)])
 def test_cache_rows_past_each_length_are_never_used(dtype, d, bs):
     """Tokens at or past a row's length (the rest of its last block and beyond)
     may hold anything: filling them with NaN changes no output bit."""
@@ -184,8 +186,11 @@ def test_cache_rows_past_each_length_are_never_used(dtype, d, bs):
     a = dw.dec.step(dw.q, dw.K, dw.V, w.n, tau=tau, tau_batch_stride=0, seq_lens=seq).clone()
     da = dw.dec.dense(dw.q, dw.K, dw.V, w.n, seq_lens=seq).clone()
     for b, n_b in enumerate(lens):
-        dw.K[b, :, n_b:] = float("nan")
-        dw.V[b, :, n_b:] = float("nan")
+        for t in (dw.K, dw.V):
+            if t.dtype == torch.float8_e4m3fn:
+                t.view(torch.uint8)[b, :, n_b:] = 0x7f       # the e4m3 NaN code
+            else:
+                t[b, :, n_b:] = float("nan")
     b_ = dw.dec.step(dw.q, dw.K, dw.V, w.n, tau=tau, tau_batch_stride=0, seq_lens=seq).clone()
     db = dw.dec.dense(dw.q, dw.K, dw.V, w.n, seq_lens=seq).clone()
     torch.cuda.synchronize()

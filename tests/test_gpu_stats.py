@@ -18,6 +18,7 @@ pytestmark = pytest.mark.gpu
     ("bf16", 8, 2, 128, 32, binding.GATE_SIGMOID),
     ("bf16", 8, 1, 64, 64, binding.GATE_SIGMOID),
     ("f32", 4, 4, 64, 16, binding.GATE_HARD),
+    ("fp8", 8, 2, 128, 32, binding.GATE_SIGMOID),
 ])
 def test_block_stats_and_diagnostics_match_oracle(dtype, Hq, Hkv, d, bs, gate):
     w = synth.Workload("stats", dtype, 2, Hq, Hkv, d, bs * 45 + 11, bs, z=1.0, tau_mode="const",
