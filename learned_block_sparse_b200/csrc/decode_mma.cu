@@ -118,21 +118,16 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// fp8 K/V. Two e4m3 bytes of w, picked by the byte permutation `sel` into bits
-// 8-15 and 24-31, become an f16x2 of the same values times 2^-8: the sign,
-// the 4 exponent bits and the 3 mantissa bits move into the f16 fields
-// unchanged, so the f16 exponent is the e4m3 one read with bias 15 instead of
-// 7. Exact for every finite e4m3 value, subnormals included; the 2^8 is put
-// back on the logits and the output.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_scaled(uint32_t w, uint32_t sel) {
-  uint32_t t;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(w), "r"(0u), "r"(sel));
-  return (t & 0x80008000u) | ((t >> 1) & 0x3f803f80u);
+// fp8 K/V: four e4m3 bytes -> two f16x2 (bytes 0,1 and bytes 2,3). Exact: every
+// e4m3 value is an f16 value. (Measured: widening the values by bit placement
+// on the integer pipe instead, to unload the conversion unit, costs more issue
+// slots than it saves: 0.59 of the copy bandwidth against 0.66.)
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo2, uint32_t& hi2) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo2), "=r"(hi2)
+      : "r"(w));
 }
-constexpr uint32_t kSelB01 = 0x1404u;  // bytes 0, 1
-constexpr uint32_t kSelB23 = 0x3424u;  // bytes 2, 3
-constexpr uint32_t kSelB02 = 0x2404u;  // bytes 0, 2
-constexpr uint32_t kSelB13 = 0x3414u;  // bytes 1, 3
 
 // As mma_rows8 / mma_16816 with f16 operands.
 __device__ __forceinline__ void mma_rows8_f16(float& d0, float& d1, uint32_t a_lo, uint32_t a_hi, uint32_t b0,
@@ -160,7 +155,8 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32
 // 2q+1 <- dims 4q, 4q+1; slots 2q+8, 2q+9 <- dims 4q+2, 4q+3) and the query
 // fragments follow the same order, which leaves every dot product unchanged.
 // For P V the transposed fragment holds two keys x two dims; the byte
-// permutation splits it into the even-dim and the odd-dim n-tile.
+// permutation splits it into the even-dim and the odd-dim n-tile. The bytes
+// become f16 in registers (exactly) and the contractions run on f16 mma.
 template <int D, int G, bool DENSE, int CH, bool HARD, bool FP8>
 __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -306,10 +302,10 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     if (live_row) {
 #pragma unroll
       for (int j = 0; j < NDT; ++j) {
-        if constexpr (FP8) {  // n-tile 2g + p holds dims 16g + 2c + p; values carry the 2^-8
+        if constexpr (FP8) {  // n-tile 2g + p holds dims 16g + 2c + p
           const int base = 16 * (j >> 1) + (j & 1);
-          s_macc[(warp * G + row) * D + base + 4 * qd] = (o[j][0] + o[j][2]) * 256.0f;
-          s_macc[(warp * G + row) * D + base + 4 * qd + 2] = (o[j][1] + o[j][3]) * 256.0f;
+          s_macc[(warp * G + row) * D + base + 4 * qd] = o[j][0] + o[j][2];
+          s_macc[(warp * G + row) * D + base + 4 * qd + 2] = o[j][1] + o[j][3];
         } else {
           s_macc[(warp * G + row) * D + 8 * j + 2 * qd] = o[j][0] + o[j][2];
           s_macc[(warp * G + row) * D + 8 * j + 2 * qd + 1] = o[j][1] + o[j][3];
@@ -332,8 +328,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     return Sv * rcp_approx(1.0f + ex2_approx(nbl * (Sv - tau_r))) * kLog2e;
   };
 
-  // fp8 keys enter the mma scaled by 2^-8 (exact): the logit scale takes it back
-  const float qscale = FP8 ? a.qscale * 256.0f : a.qscale;
+  const float qscale = a.qscale;
   auto process = [&](int st, const int4 inf) {
     const uint32_t kt = smem_u32(s_tiles + static_cast<size_t>(st) * 2 * tile_bytes);
     const uint32_t vt = kt + tile_bytes;
@@ -361,8 +356,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
           for (int m = 0; m < 4; ++m)
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
-              const uint32_t b0 = e4m3x2_to_f16x2_scaled(bb[j][m], kSelB01);
-              const uint32_t b1 = e4m3x2_to_f16x2_scaled(bb[j][m], kSelB23);
+              uint32_t b0, b1;  // dims 4q, 4q+1 and 4q+2, 4q+3 of the key
+              e4m3x4_to_f16x2x2(bb[j][m], b0, b1);
               if (m & 1) mma_rows8_f16(so[j][0], so[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
               else mma_rows8_f16(se[j][0], se[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
             }
@@ -456,14 +451,22 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
           for (int g = 0; g < D / 16; g += 2) {
             uint32_t r0, r1, r2, r3;
             ldsm_x4_t(vt + swz(bs, vrow, g + (lane >> 4)), r0, r1, r2, r3);
-            mma_16816_f16(o[2 * g], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r0, kSelB02),
-                          e4m3x2_to_f16x2_scaled(r1, kSelB02));
-            mma_16816_f16(o[2 * g + 1], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r0, kSelB13),
-                          e4m3x2_to_f16x2_scaled(r1, kSelB13));
-            mma_16816_f16(o[2 * g + 2], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r2, kSelB02),
-                          e4m3x2_to_f16x2_scaled(r3, kSelB02));
-            mma_16816_f16(o[2 * g + 3], h0, l0, h1, l1, e4m3x2_to_f16x2_scaled(r2, kSelB13),
-                          e4m3x2_to_f16x2_scaled(r3, kSelB13));
+            // each register: keys 2q, 2q+1 x dims 2c, 2c+1; regroup into the
+            // even-dim and the odd-dim key pairs (bytes 0,2 and 1,3)
+            uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
+            auto split = [](uint32_t r, uint32_t& ev, uint32_t& od) {
+              uint32_t t;
+              asm("prmt.b32 %0, %1, %2, %3;" : "=r"(t) : "r"(r), "r"(0u), "r"(0x3120u));
+              e4m3x4_to_f16x2x2(t, ev, od);
+            };
+            split(r0, e0, o0);
+            split(r1, e1, o1);
+            split(r2, e2, o2);
+            split(r3, e3, o3);
+            mma_16816_f16(o[2 * g], h0, l0, h1, l1, e0, e1);
+            mma_16816_f16(o[2 * g + 1], h0, l0, h1, l1, o0, o1);
+            mma_16816_f16(o[2 * g + 2], h0, l0, h1, l1, e2, e3);
+            mma_16816_f16(o[2 * g + 3], h0, l0, h1, l1, o2, o3);
           }
         } else {
           const uint32_t h0 = pack_bf16x2(p[2 * m2][0], p[2 * m2][1]);
