@@ -336,3 +336,16 @@ def test_full_size_512k_sampled():
 def test_full_size_64k_b16_batch16_sampled():
     w = synth.WORKLOADS[5].replace(B=16)
     _full_size(w, 0.25, 0, list_pairs=[(0, 0), (9, 3), (15, 15)])
+
+
+def test_full_size_fp8_gqa_128k():
+    """Workload 7 (the 128K GQA workload with fp8 K/V) at full size."""
+    w = synth.WORKLOADS[7]
+    dens = _full_size(w, 0.38, 0, list_pairs=[(0, 0), (5, 3), (7, 7)])
+    assert 0.3 < dens < 0.5
+
+
+def test_full_size_table10_shape_sampled():
+    """The pages' Table 10 head shape (32/4 heads, d 64, b 64) at 512K tokens, batch 4."""
+    w = synth.WORKLOADS[6].replace(B=4)
+    _full_size(w, 0.05, 0, list_pairs=[(0, 0), (3, 3)])
