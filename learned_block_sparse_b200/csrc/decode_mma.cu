@@ -35,15 +35,18 @@ namespace eta {
 
 namespace {
 
-// Consumer warps: 4, or 8 where a block carries more consumer work per byte
-// than a 32-token bf16 block at d=128: 16-token blocks (half the bytes per
-// block for the same fixed cost), d=64 (twice the keys, hence twice the gate
-// and softmax work, per byte) and fp8 K/V (half the bytes, plus the
-// conversions); plus one producer warp.
+// Consumer warps, plus one producer warp. A warp owns a whole block and its
+// per-block chain (QK^T, gate, softmax, PV) is latency-bound, so the warp count
+// sets how many blocks are in work per SM: 6 for 32-key chunks at d=128 (4
+// warps held the 128K GQA decode at 0.99 of the copy bandwidth, 6 reach 1.09),
+// 8 where a block carries more consumer work per byte: 16-token blocks,
+// d=64 (twice the keys per byte) and fp8 K/V (half the bytes, plus the
+// conversions), whose kernels fit 168 registers.
 template <int D, int CH, bool FP8>
 struct MmaWarps {
-  static constexpr int kMW = (CH == 16 || D == 64 || FP8) ? 8 : 4;
+  static constexpr int kMW = (CH == 16 || D == 64 || FP8) ? 8 : 6;
   static constexpr int kThreads = (kMW + 1) * 32;
+  static constexpr int kIssueLanes = kMW >= 8 ? 8 : 4;  // producer lanes (a power of two)
 };
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar,
@@ -253,7 +256,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&s_full[st]);
     };
-    producer_loop<G, DENSE, kMW>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of, pre, issue, s_full);
+    producer_loop<G, DENSE, MmaWarps<D, CH, FP8>::kIssueLanes>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of,
+                                                               pre, issue, s_full);
     return;
   }
 
