@@ -98,12 +98,34 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // device status word are set) or when another thread of the CTA has aborted.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// Bounded wait until the shared int *p equals v (set by another warp of the
+// thread block); same limit and abort protocol as mbar_wait_bounded below.
+__device__ __forceinline__ bool wait_value_bounded(volatile int* p, int v, volatile int* abort_flag,
+                                                   int32_t* status);
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                   int32_t* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicExch(status, static_cast<int32_t>(ETA_ERR_DEVICE_TIMEOUT));
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_value_bounded(volatile int* p, int v, volatile int* abort_flag,
+                                                   int32_t* status) {
+  if (*p == v) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (*p == v) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {

@@ -178,11 +178,13 @@ __device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int
 // of the K and V stores), which must arm s_full[stage] (arrive +
 // expected bytes) and start the copies. The warp reads the union list 32
 // entries at a time, one batch ahead. A stage's r-th reuse waits for the
-// consumer release that completed the empty barrier's phase r-1.
+// consumer release that completed the empty barrier's phase r-1; the round a
+// stage serves is then published in s_round (when given) before it is armed.
 template <int G, bool DENSE, int kMaxPL, typename SegOf, typename Pre, typename Issue>
 __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, int64_t hi, int NST,
                                               uint64_t* s_empty, int4* s_info, int* s_abort, SegOf seg_of,
-                                              Pre pre, Issue issue, uint64_t* s_full) {
+                                              Pre pre, Issue issue, uint64_t* s_full,
+                                              volatile int* s_round = nullptr) {
   static_assert(kMaxPL == 1 || kMaxPL == 2 || kMaxPL == 4 || kMaxPL == 8, "issuing lanes divide 32");
   int PL = kMaxPL;  // issuing lanes
   while (PL > NST) PL >>= 1;
@@ -242,6 +244,7 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
             atomicExch(a.status, static_cast<int32_t>(ETA_ERR_INVALID_ARG));
             rows = 0;
           }
+          if (s_round != nullptr) s_round[st] = round;  // this stage now serves round `round`
           s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
           if (rows == 0) mbar_arrive(&s_full[st]);
           else issue(st, row_i, rows);

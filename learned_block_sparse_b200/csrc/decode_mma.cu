@@ -185,7 +185,8 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
   uint64_t* s_empty = s_full + NST;
   uint64_t* s_aux = s_empty + NST;  // [8] per issuing lane: copies of a partial block
   int4* s_info = reinterpret_cast<int4*>(s_aux + 8);
-  float* s_macc = reinterpret_cast<float*>(s_info + NST);  // [kMW][G][D]
+  int* s_round = reinterpret_cast<int*>(s_info + NST);     // [NST] round each stage serves
+  float* s_macc = reinterpret_cast<float*>(s_round + NST); // [kMW][G][D]
   float* s_mm = s_macc + kMW * G * D;                      // [kMW][G]
   float* s_ml = s_mm + kMW * G;                            // [kMW][G]
   int* s_abort = reinterpret_cast<int*>(s_ml + kMW * G);
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
       mbar_init(&s_empty[s], 1);
     }
     for (int s = 0; s < 8; ++s) mbar_init(&s_aux[s], 1);
+    for (int s = 0; s < NST; ++s) s_round[s] = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
       mbar_arrive(&s_full[st]);
     };
     producer_loop<G, DENSE, MmaWarps<D, CH, FP8>::kIssueLanes>(a, lo, hi, NST, s_empty, s_info, s_abort, seg_of,
-                                                               pre, issue, s_full);
+                                                               pre, issue, s_full, s_round);
     return;
   }
 
@@ -517,14 +519,15 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     const int st = it % NST;
     const int round = it / NST;
     // Consecutive uses of a stage belong to different warps, so this warp may
-    // get here before the stage's previous use has even landed; an mbarrier
-    // wait on a phase two ahead of the current one would return at once. Wait
-    // for the previous use's release first: then the full barrier is at most
-    // one phase behind and the parity wait below is exact.
-    // (With a stage count that is a multiple of kMW a stage always returns to
-    // the same warp, which has released it itself, and the extra wait is skipped.)
-    bool ok = round == 0 || (NST % kMW) == 0 ||
-              mbar_wait_bounded(&s_empty[st], static_cast<uint32_t>((round - 1) & 1), s_abort, a.status);
+    // get here rounds ahead of the stage (with fewer stages than warps, even
+    // before the round before it has been released), and an mbarrier parity
+    // wait on a phase two or more ahead returns at once. Wait until the
+    // producer has published this round for the stage: it does so only after
+    // the previous round's release, so the full barrier is then in this round's
+    // phase and the parity wait below is exact. (With a stage count that is a
+    // multiple of kMW a stage always returns to the same warp, which released
+    // it itself, and the extra wait is skipped.)
+    bool ok = round == 0 || (NST % kMW) == 0 || wait_value_bounded(s_round + st, round, s_abort, a.status);
     ok = ok && mbar_wait_bounded(&s_full[st], static_cast<uint32_t>(round & 1), s_abort, a.status);
     if (ok) process(st, s_info[st]);
     __syncwarp();
@@ -569,7 +572,7 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   constexpr unsigned kThreads = MmaWarps<D, CH, FP8>::kThreads;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 + 8 * sizeof(uint64_t) +
                        static_cast<size_t>(BH + 1) * sizeof(int32_t) + 1024;
-  const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4);
+  const size_t per_stage = 2 * tile + 2 * sizeof(uint64_t) + sizeof(int4) + sizeof(int);
   const size_t budget = static_cast<size_t>(device_max_smem_optin()) - 512;
   if (fixed + 2 * per_stage > budget) return cudaErrorInvalidValue;
   // ~200 KB of stages: the consumer warps hold up to kMW, the rest are in flight.

@@ -135,12 +135,17 @@ def test_dtypes_dims_blocks(dtype, d, bs):
     _full_check(w, dense=True)
 
 
-@pytest.mark.parametrize("bs,n_splits", [(64, 2), (64, 5), (128, 3), (32, 4), (16, 3)])
-def test_long_ranges_reuse_every_stage_many_times(bs, n_splits):
+@pytest.mark.parametrize("dtype,d,bs,n_splits", [
+    ("bf16", 128, 64, 2), ("bf16", 128, 64, 5), ("bf16", 128, 128, 3), ("bf16", 128, 32, 4), ("bf16", 128, 16, 3),
+    # rings with fewer stages than consumer warps (3 < 6, 6 < 8) and stage counts
+    # that are not multiples of the warp count
+    ("bf16", 128, 128, 1), ("bf16", 64, 128, 2), ("fp8", 128, 128, 2), ("bf16", 64, 64, 3), ("fp8", 128, 64, 3),
+])
+def test_long_ranges_reuse_every_stage_many_times(dtype, d, bs, n_splits):
     """Few split ranges, so each thread block streams hundreds of blocks through
     its ring and every stage is reused many times by different consumer warps."""
-    w = synth.Workload("ring", "bf16", 1, 4, 4, 128, bs * 700 + 3, bs, z=1.0, tau_mode="const",
-                       densities=(0.5,), seed=bs + n_splits, offset_std=synth.SQRT_HALF)
+    w = synth.Workload("ring", dtype, 1, 4, 4, d, bs * 700 + 3, bs, z=1.0, tau_mode="const",
+                       densities=(0.5,), seed=bs + n_splits + d, offset_std=synth.SQRT_HALF)
     _full_check(w, 0.5, n_splits=n_splits, dense=True)
 
 
