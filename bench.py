@@ -486,7 +486,7 @@ def run_eta(args):
         "metric": "sparse decode queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8": "fp8", "f32": "f32"}[w.dtype],
-        "data": "synthetic (seeded Philox4x32-10 + Box-Muller; see DESIGN.md input recipe)",
+        "data": "synthetic (seeded Philox4x32-10 + Box-Muller normals, shaped like the pages' decode workloads)",
         "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
                    "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
                    "l2": ("flushed before every timed step: 512 MiB write" +
