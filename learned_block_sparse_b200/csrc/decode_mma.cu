@@ -44,7 +44,7 @@ namespace {
 // conversions), whose kernels fit 168 registers.
 template <int D, int CH, bool FP8>
 struct MmaWarps {
-  static constexpr int kMW = (CH == 16 || D == 64 || FP8) ? 8 : 6;
+  static constexpr int kMW = (CH == 16 || D == 64) ? 8 : (FP8 ? 7 : 6);
   static constexpr int kThreads = (kMW + 1) * 32;
   static constexpr int kIssueLanes = kMW >= 8 ? 8 : 4;  // producer lanes (a power of two)
 };
@@ -132,16 +132,42 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo2, uin
       : "r"(w));
 }
 
-// As mma_rows8 / mma_16816 with f16 operands.
-__device__ __forceinline__ void mma_rows8_f16(float& d0, float& d1, uint32_t a_lo, uint32_t a_hi, uint32_t b0,
-                                              uint32_t b1) {
-  [[maybe_unused]] float z2, z3;
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %10, %11};"
-      : "+f"(d0), "+f"(d1), "=f"(z2), "=f"(z3)
-      : "r"(a_lo), "r"(0u), "r"(a_hi), "r"(0u), "r"(b0), "r"(b1), "f"(0.0f), "f"(0.0f));
+// Two floats -> two e4m3 bytes (lo in bits 0-7), rounded to nearest even,
+// saturating at +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
 }
+
+// Four floats (|v| < 256) -> a high and a low e4m3 word with v = hi + lo / 16:
+// hi keeps the top four significant bits of each value and lo the next four,
+// so a bf16 value (eight significant bits) is held exactly unless its low part
+// falls below the e4m3 subnormal step (values under 2^-6 of the largest one).
+__device__ __forceinline__ void e4m3_split4(float v0, float v1, float v2, float v3, uint32_t& hi, uint32_t& lo) {
+  const uint32_t h = f32x2_to_e4m3x2(v0, v1) | (f32x2_to_e4m3x2(v2, v3) << 16);
+  uint32_t f01, f23;
+  e4m3x4_to_f16x2x2(h, f01, f23);
+  const float2 b01 = __half22float2(*reinterpret_cast<const __half2*>(&f01));
+  const float2 b23 = __half22float2(*reinterpret_cast<const __half2*>(&f23));
+  hi = h;
+  lo = f32x2_to_e4m3x2((v0 - b01.x) * 16.0f, (v1 - b01.y) * 16.0f) |
+       (f32x2_to_e4m3x2((v2 - b23.x) * 16.0f, (v3 - b23.y) * 16.0f) << 16);
+}
+
+// D[16x8] += A[16x32] B[32x8], e4m3 in, fp32 accumulate. Byte i of a0 / a2 is
+// A[lane/4][4(lane%4) + i] / A[lane/4][16 + 4(lane%4) + i], a1 / a3 the same
+// for row lane/4 + 8; byte i of b0 / b1 is B[4(lane%4) + i][lane/4] /
+// B[16 + 4(lane%4) + i][lane/4].
+__device__ __forceinline__ void mma_16832_e4m3(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// As mma_16816 with f16 operands.
 __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                               uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -152,14 +178,16 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32
 }
 
 // HARD: the strict-mode gate (keys below tau removed) instead of Eq. 2-3.
-// FP8: e4m3 K/V (d = 128). A 16-byte shared chunk then holds 16 dims of one
-// key, so an ldmatrix fragment gives a thread dims 4q..4q+3 of one key (q =
-// lane % 4); the k slots of the f16 mma take them in that order (slots 2q,
-// 2q+1 <- dims 4q, 4q+1; slots 2q+8, 2q+9 <- dims 4q+2, 4q+3) and the query
-// fragments follow the same order, which leaves every dot product unchanged.
+// FP8: e4m3 K/V (d = 128). Q K^T runs on e4m3 mma (m16n8k32) straight from the
+// key bytes: an ldmatrix fragment of a 16-byte chunk gives a thread dims
+// 4q..4q+3 of one key (q = lane % 4), which is the e4m3 B-operand layout. The
+// query, bf16, is scaled per head by a power of two (its largest |q| into
+// [128, 256)) and split into a high and a low e4m3 term (q = hi + lo/16, exact
+// for bf16): the high terms are A rows 0-7 and the low terms rows 8-15, so one
+// mma gives both partial products of a key and S = (hi + lo/16) * scale.
 // For P V the transposed fragment holds two keys x two dims; the byte
-// permutation splits it into the even-dim and the odd-dim n-tile. The bytes
-// become f16 in registers (exactly) and the contractions run on f16 mma.
+// permutation splits it into the even-dim and the odd-dim n-tile, whose bytes
+// become f16 in registers (exactly) for an f16 mma with the f16 P.
 template <int D, int G, bool DENSE, int CH, bool HARD, bool FP8>
 __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     decode_mma_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap tmk,
@@ -266,7 +294,9 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
   // -------------------------------------------------------------- consumers
   const int row = lane >> 2, qd = lane & 3;
   const bool live_row = row < G;
-  uint32_t qa[KST][2];
+  uint32_t qa[KST][2];  // bf16 query fragments of the k16 steps
+  uint32_t q8[4][4];    // fp8: e4m3 query fragments of the k32 steps (rows 8-15: low terms)
+  float qs_r = a.qscale;  // fp8: 1/sqrt(d) over this head's query scale
   float o[NDT][4];  // [n-tile][c0 c1 = high part of row, c2 c3 = low part]
   float m_r = -INFINITY, l_r = 0.0f, tau_r = 0.0f;
   int64_t t_cur = 0;  // position of the current token of the segment being attended
@@ -274,21 +304,41 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
   auto load_q = [&](int seg) {
     const int b = seg / a.Hkv, kvh = seg % a.Hkv;
     t_cur = seg_tokens(a, seg) - 1;
-    if (live_row) {
+    if constexpr (FP8) {
+      const uint16_t* qp =
+          static_cast<const uint16_t*>(a.q) + (static_cast<int64_t>(b) * a.Hq + kvh * G + (live_row ? row : 0)) * D;
+      tau_r = live_row ? (a.tau != nullptr ? a.tau[b * a.tau_stride + kvh * G + row] : -INFINITY) : 0.0f;
+      // this thread's dims of k32 step kk: 32kk + 4qd + i (i < 4), then 16 more
+      float x[4][8];
+      float amax = 0.0f;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int c = 32 * kk + 16 * (i >> 2) + 4 * qd + (i & 3);
+          x[kk][i] = live_row ? __uint_as_float(static_cast<uint32_t>(qp[c]) << 16) : 0.0f;
+          amax = fmaxf(amax, fabsf(x[kk][i]));
+        }
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 2));
+      // 2^e with 2^e * amax in [128, 256) (amax = 2^(E-127) * 1.f)
+      const int E = (__float_as_int(amax) >> 23) & 0xff;
+      const int e = E == 0 ? 0 : max(-120, min(120, 134 - E));
+      const float up = __int_as_float((127 + e) << 23);
+      qs_r = a.qscale * __int_as_float((127 - e) << 23);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        e4m3_split4(x[kk][0] * up, x[kk][1] * up, x[kk][2] * up, x[kk][3] * up, q8[kk][0], q8[kk][1]);
+        e4m3_split4(x[kk][4] * up, x[kk][5] * up, x[kk][6] * up, x[kk][7] * up, q8[kk][2], q8[kk][3]);
+      }
+    } else if (live_row) {
       const uint16_t* qp =
           static_cast<const uint16_t*>(a.q) + (static_cast<int64_t>(b) * a.Hq + kvh * G + row) * D;
 #pragma unroll
       for (int kk = 0; kk < KST; ++kk) {
-        if constexpr (FP8) {  // f16 fragments in the key fragments' dim order (see the kernel comment)
-          const int c = 16 * kk + 4 * qd;
-          auto f = [&](int i) { return __uint_as_float(static_cast<uint32_t>(qp[c + i]) << 16); };
-          qa[kk][0] = pack_f16x2(f(0), f(1));
-          qa[kk][1] = pack_f16x2(f(2), f(3));
-        } else {
-          const int c = 16 * kk + 2 * qd;
-          qa[kk][0] = static_cast<uint32_t>(qp[c]) | (static_cast<uint32_t>(qp[c + 1]) << 16);
-          qa[kk][1] = static_cast<uint32_t>(qp[c + 8]) | (static_cast<uint32_t>(qp[c + 9]) << 16);
-        }
+        const int c = 16 * kk + 2 * qd;
+        qa[kk][0] = static_cast<uint32_t>(qp[c]) | (static_cast<uint32_t>(qp[c + 1]) << 16);
+        qa[kk][1] = static_cast<uint32_t>(qp[c + 8]) | (static_cast<uint32_t>(qp[c + 9]) << 16);
       }
       tau_r = a.tau != nullptr ? a.tau[b * a.tau_stride + kvh * G + row] : -INFINITY;
     } else {
@@ -346,29 +396,35 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     constexpr int NT = CH / 8;  // n-tiles of 8 keys per chunk
     for (int c0 = 0; c0 < bs; c0 += CH) {
       // S = Q K^T: even and odd k-steps accumulate separately (shorter mma chains)
-      float se[NT][2], so[NT][2];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) se[j][0] = se[j][1] = so[j][0] = so[j][1] = 0.0f;
+      float se[NT][2], so[NT][2];  // bf16: partial sums of the even and odd k-steps
+      float sv[FP8 ? NT : 1][2];   // fp8: the scaled logits
       if constexpr (FP8) {
-        // a 16-byte chunk is one k-step: an x4 load gives 4 k-steps of one n-tile
+        // two 16-byte chunks are one k32 step: an x4 load gives 2 k-steps of one n-tile
+        float sa[NT][4], sb[NT][4];
 #pragma unroll
-        for (int k4 = 0; k4 < KST / 4; ++k4) {
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) sa[j][r] = sb[j][r] = 0.0f;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
           uint32_t bb[NT][4];
 #pragma unroll
           for (int j = 0; j < NT; ++j)
-            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k4 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * u + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
                     bb[j][3]);
 #pragma unroll
-          for (int m = 0; m < 4; ++m)
+          for (int j = 0; j < NT; ++j) mma_16832_e4m3(sa[j], q8[2 * u], bb[j][0], bb[j][1]);
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-              uint32_t b0, b1;  // dims 4q, 4q+1 and 4q+2, 4q+3 of the key
-              e4m3x4_to_f16x2x2(bb[j][m], b0, b1);
-              if (m & 1) mma_rows8_f16(so[j][0], so[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
-              else mma_rows8_f16(se[j][0], se[j][1], qa[4 * k4 + m][0], qa[4 * k4 + m][1], b0, b1);
-            }
+          for (int j = 0; j < NT; ++j) mma_16832_e4m3(sb[j], q8[2 * u + 1], bb[j][2], bb[j][3]);
         }
+        // rows 0-7 hold the high-term products, rows 8-15 the low-term ones
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) sv[j][e] = fmaf(sa[j][2 + e] + sb[j][2 + e], 0.0625f, sa[j][e] + sb[j][e]) * qs_r;
       } else {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) se[j][0] = se[j][1] = so[j][0] = so[j][1] = 0.0f;
 #pragma unroll
         for (int k2 = 0; k2 < KST / 2; ++k2) {
           uint32_t bb[NT][4];
@@ -384,6 +440,10 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
             mma_rows8(so[j][0], so[j][1], qa[2 * k2 + 1][0], qa[2 * k2 + 1][1], bb[j][2], bb[j][3]);
         }
       }
+      auto s_at = [&](int j, int e) {  // scaled logit of key 8j + 2qd + e of the chunk
+        if constexpr (FP8) return sv[j][e];
+        else return (se[j][e] + so[j][e]) * qscale;
+      };
       // gate (Eq. 2-3) and online softmax on this thread's row
       float g[NT][2];
       float bm = -INFINITY;
@@ -392,7 +452,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
         for (int j = 0; j < NT; ++j)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float v = row_on ? gate((se[j][e] + so[j][e]) * qscale) : -INFINITY;
+            const float v = row_on ? gate(s_at(j, e)) : -INFINITY;
             g[j][e] = v;
             bm = fmaxf(bm, v);
           }
@@ -404,7 +464,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
             const int key = c0 + 8 * j + 2 * qd + e;
             float v = -INFINITY;
             if (row_on && key < rows) {
-              const float Sv = (se[j][e] + so[j][e]) * qscale;
+              const float Sv = s_at(j, e);
               // the current token is exempt from the gate (Eq. 3)
               v = (tok0 + key == t_cur) ? Sv * kLog2e : gate(Sv);
             }
@@ -622,8 +682,8 @@ cudaError_t launch_mma_g(const DecodeCall& c, cudaStream_t st) {
 // conversions need the registers of the second half-chunk).
 template <int D, bool DENSE, bool FP8>
 cudaError_t launch_mma_c(const DecodeCall& c, cudaStream_t st) {
-  if (FP8 || c.shape.block_size == 16) return launch_mma_g<D, DENSE, 16, FP8>(c, st);
-  return launch_mma_g<D, DENSE, (FP8 ? 16 : 32), FP8>(c, st);
+  if (c.shape.block_size == 16) return launch_mma_g<D, DENSE, 16, FP8>(c, st);
+  return launch_mma_g<D, DENSE, 32, FP8>(c, st);
 }
 
 }  // namespace

@@ -256,12 +256,13 @@ def test_thresholds_in_screen_equal_separate_predictor(dtype, G, bs):
     assert torch.equal(fused, sep)
 
 
-@pytest.mark.parametrize("dtype,G,bs", [("bf16", 4, 32), ("bf16", 8, 64), ("f32", 1, 16), ("bf16", 1, 16)])
+@pytest.mark.parametrize("dtype,G,bs", [("bf16", 4, 32), ("bf16", 8, 64), ("f32", 1, 16), ("bf16", 1, 16),
+                                        ("fp8", 4, 32), ("fp8", 8, 16)])
 def test_strict_mode_gate(dtype, G, bs):
     """Strict mode (keys below tau removed): lists and outputs against the oracle.
     Each head's tau sits in a wide gap of its own true logits, so the keep/remove
     decision does not depend on how either side rounds S."""
-    d = 64 if (G == 8 or dtype == "f32") else 128
+    d = 128 if dtype == "fp8" else (64 if (G == 8 or dtype == "f32") else 128)
     w = synth.Workload("strict", dtype, 2, 2 * G, 2, d, bs * 60 + 5, bs, z=1.0, tau_mode="const",
                        densities=(0.5,), seed=300 + G + bs, offset_std=synth.SQRT_HALF)
     dw = DeviceWorkload(w, keep_host=True, gate=binding.GATE_HARD)
