@@ -61,6 +61,8 @@ def lib():
         L.oracle_inv_sqrt_d.restype = f32
         L.oracle_screen_head.argtypes = [vp, i32, vp, vp, vp, i64, i32, f32, f32, f32, vp, vp]
         L.oracle_screen_head.restype = i32
+        L.oracle_screen_head_env.argtypes = [vp, i32, vp, vp, vp, i64, i32, i32, f32, f32, f32, vp, vp]
+        L.oracle_screen_head_env.restype = i32
         L.oracle_attend_head.argtypes = [i32, vp, vp, i32, i32, i64, vp, vp, i32, f32, f32, i32, vp]
         L.oracle_block_stats.argtypes = [i32, vp, i32, i32, i64, i32, vp, f32, f32, f32, i32, vp, vp, vp]
         for fn in ("oracle_to_f32", "oracle_block_meta", "oracle_slice_meta",
@@ -185,6 +187,27 @@ def screen_head(q_f32, mu, var, maxn, nb: int, n_local: int, z: float, tau: floa
     sc = np.zeros((max(ns, 1),), np.float32)
     cnt = lib().oracle_screen_head(_p(q_f32), d, _p(mu), _p(var), _p(maxn), nb, n_local,
                                    float(z), float(tau), float(offset_a), _p(lst), _p(sc))
+    return lst[:cnt].copy(), sc[:ns].copy()
+
+
+def screen_head_env(q_f32, mu, var, maxn, nb: int, r: int, n_local: int, z: float, tau: float,
+                    offset_a: float = 0.0):
+    """Sub-block envelope screen of one head (a labelled reading of the pages'
+    undefined "sub-block envelope"): mu, var [>= ns*r][d] and maxn [>= ns*r] are
+    the metadata of sub-blocks of b/r tokens; a block's score is the largest of
+    its r sub-block scores (Eq. 5 on each). Returns the admitted ascending block
+    list and the envelope scores of the screened blocks."""
+    q_f32 = np.ascontiguousarray(q_f32, np.float32)
+    d = q_f32.shape[0]
+    mu = np.ascontiguousarray(mu, np.float32)
+    var = np.ascontiguousarray(var, np.float32)
+    maxn = np.ascontiguousarray(maxn, np.float32)
+    ns = max(0, nb - n_local)
+    assert mu.shape[0] >= ns * r and maxn.shape[0] >= ns * r
+    lst = np.zeros((max(nb, 1),), np.int32)
+    sc = np.zeros((max(ns, 1),), np.float32)
+    cnt = lib().oracle_screen_head_env(_p(q_f32), d, _p(mu), _p(var), _p(maxn), nb, int(r), n_local,
+                                       float(z), float(tau), float(offset_a), _p(lst), _p(sc))
     return lst[:cnt].copy(), sc[:ns].copy()
 
 

@@ -173,6 +173,42 @@ int oracle_screen_head(const float* q, int d, const float* mu, const float* var,
   return cnt;
 }
 
+/*
+ * Sub-block envelope (a labelled reading): the pages name a "sub-block
+ * envelope" as the remedy for variance dilution under flat block variance
+ * (Table 16 caption; Table 12's 1.45B header, b = 64) without defining it.
+ * Reading taken here: each block of b tokens is split into r = b / b_s
+ * sub-blocks of b_s consecutive tokens, each with its own metadata (mean,
+ * population variance, largest key norm, as for a block of b_s tokens); the
+ * block's score is the largest of its r sub-block scores (Eq. 5 on each
+ * sub-block), i.e. the upper envelope, and the admission rule is unchanged.
+ * r = 1 is Eq. 5 as printed.
+ *   mu, var : [>= ns*r][d], maxn : [>= ns*r] sub-block metadata
+ *   list    : [nb] out, ascending admitted block indices; returns the count
+ *   scores  : [ns] out (may be NULL), the envelope score of each screened block
+ */
+int oracle_screen_head_env(const float* q, int d, const float* mu, const float* var,
+                           const float* maxn, int64_t nb, int r, int n_local, float z,
+                           float tau, float offset_a, int32_t* list, float* scores) {
+  const float s = oracle_inv_sqrt_d(d);
+  const float tau_t = tau - offset_a;
+  int64_t ns = nb - n_local;
+  if (ns < 0) ns = 0;
+  int cnt = 0;
+  for (int64_t j = 0; j < ns; ++j) {
+    float env = -INFINITY;
+    for (int u = 0; u < r; ++u) {
+      const int64_t sb = j * r + u;
+      const float sc = oracle_block_score(q, d, mu + sb * d, var + sb * d, maxn[sb], z, s);
+      if (sc > env) env = sc;
+    }
+    if (scores) scores[j] = env;
+    if (!(env < tau_t)) list[cnt++] = (int32_t)j;
+  }
+  for (int64_t j = ns; j < nb; ++j) list[cnt++] = (int32_t)j;
+  return cnt;
+}
+
 static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
 
 /*
