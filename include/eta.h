@@ -44,7 +44,7 @@
 extern "C" {
 #endif
 
-#define ETA_ABI_VERSION 2
+#define ETA_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define ETA_API __attribute__((visibility("default")))
@@ -95,7 +95,21 @@ typedef struct {
                           exempts) */
   int32_t n_splits;    /* decode work ranges (thread blocks); 0 = one per SM */
   int32_t gate;        /* ETA_GATE_SIGMOID (Eq. 2-3) or ETA_GATE_HARD (strict mode) */
+  int32_t sub_blocks;  /* r: 0 or 1 = Eq. 5 on whole blocks; 2, 4 or 8 = the
+                          sub-block envelope (see below) */
 } eta_params_t;
+
+/* Sub-block envelope. The pages name a "sub-block envelope" as the remedy for
+ * variance dilution under flat block variance (Table 16 caption; Table 12's
+ * header for the 1.45B model at b = 64) and do not define it. Reading taken
+ * here: with sub_blocks = r > 1 every block of b tokens is seen as r
+ * sub-blocks of b/r consecutive tokens, each with its own metadata; a block's
+ * score is the largest Eq. 5 score of its sub-blocks and the admission rule is
+ * unchanged. The metadata arrays then hold capacity / (b/r) columns per
+ * (batch row, kv head), built by eta_build_block_meta called with a shape
+ * whose block_size is b/r over sub-block ranges. Requires b/r >= 16; not
+ * available for paged stores (ETA_ERR_UNSUPPORTED). The scores output holds
+ * the envelope score per block. */
 
 /* Logit gate of the decode (the current token t is exempt from both):
  * ETA_GATE_SIGMOID  g_s = S_s * sigmoid(beta (S_s - tau))   (Eq. 2-3; the pages'

@@ -39,7 +39,8 @@ GATE_SIGMOID, GATE_HARD = 0, 1   # Eq. 2-3 multiplicative gate; strict mode (har
 
 class Params(ctypes.Structure):
     _fields_ = [("beta", ctypes.c_float), ("z", ctypes.c_float), ("offset_a", ctypes.c_float),
-                ("n_local", ctypes.c_int32), ("n_splits", ctypes.c_int32), ("gate", ctypes.c_int32)]
+                ("n_local", ctypes.c_int32), ("n_splits", ctypes.c_int32), ("gate", ctypes.c_int32),
+                ("sub_blocks", ctypes.c_int32)]
 
 
 class Meta(ctypes.Structure):
@@ -160,8 +161,8 @@ def make_shape(batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity, kv_
                  _dtype_code(q_dtype) if isinstance(q_dtype, torch.dtype) else q_dtype)
 
 
-def make_params(beta=5.0, z=1.0, offset_a=0.0, n_local=1, n_splits=0, gate=GATE_SIGMOID) -> Params:
-    return Params(beta, z, offset_a, n_local, n_splits, gate)
+def make_params(beta=5.0, z=1.0, offset_a=0.0, n_local=1, n_splits=0, gate=GATE_SIGMOID, sub_blocks=1) -> Params:
+    return Params(beta, z, offset_a, n_local, n_splits, gate, sub_blocks)
 
 
 def build_block_meta(shape: Shape, k: torch.Tensor, blk_begin: int, blk_end: int, mu: torch.Tensor,
@@ -371,11 +372,15 @@ class EtaDecoder:
 
     def __init__(self, batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity,
                  kv_dtype=torch.bfloat16, q_dtype=torch.bfloat16, beta=5.0, z=1.0, offset_a=0.0,
-                 n_local=1, n_splits=0, device="cuda", gate=GATE_SIGMOID):
+                 n_local=1, n_splits=0, device="cuda", gate=GATE_SIGMOID, sub_blocks=1):
         self.shape = make_shape(batch, n_q_heads, n_kv_heads, head_dim, block_size, capacity, kv_dtype, q_dtype)
-        self.params = make_params(beta, z, offset_a, n_local, n_splits, gate)
+        self.params = make_params(beta, z, offset_a, n_local, n_splits, gate, sub_blocks)
         self.device = torch.device(device)
-        nb_cap = capacity // block_size
+        # the sub-block envelope keeps metadata per sub-block of block_size / sub_blocks tokens
+        self.sub_blocks = max(1, sub_blocks)
+        self.meta_shape = make_shape(batch, n_q_heads, n_kv_heads, head_dim, block_size // self.sub_blocks, capacity,
+                                     kv_dtype, q_dtype)
+        nb_cap = capacity // block_size * self.sub_blocks
         f = dict(dtype=torch.float32, device=self.device)
         self.mu = torch.zeros((batch, n_kv_heads, head_dim, nb_cap), **f)
         self.var = torch.zeros((batch, n_kv_heads, head_dim, nb_cap), **f)
@@ -389,7 +394,10 @@ class EtaDecoder:
         return (self.mu, self.var, self.maxnorm)
 
     def build_meta(self, k: torch.Tensor, blk_begin: int, blk_end: int) -> None:
-        build_block_meta(self.shape, k, blk_begin, blk_end, self.mu, self.var, self.maxnorm)
+        """Metadata of blocks [blk_begin, blk_end) (of every sub-block in them
+        with the envelope)."""
+        r = self.sub_blocks
+        build_block_meta(self.meta_shape, k, blk_begin * r, blk_end * r, self.mu, self.var, self.maxnorm)
 
     def predict_tau(self, q: torch.Tensor, W: torch.Tensor, bias: torch.Tensor) -> torch.Tensor:
         predict_tau(self.shape, q, W, bias, self.tau)

@@ -117,6 +117,18 @@ eta_status_t check_params(const eta_params_t* p) {
   if (!std::isfinite(p->z) || !std::isfinite(p->offset_a)) return ETA_ERR_INVALID_ARG;
   if (p->n_local < 1 || p->n_splits < 0) return ETA_ERR_INVALID_ARG;
   if (p->gate != ETA_GATE_SIGMOID && p->gate != ETA_GATE_HARD) return ETA_ERR_INVALID_ARG;
+  if (p->sub_blocks != 0 && p->sub_blocks != 1 && p->sub_blocks != 2 && p->sub_blocks != 4 && p->sub_blocks != 8)
+    return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+int sub_blocks_of(const eta_params_t* p) { return p->sub_blocks > 1 ? p->sub_blocks : 1; }
+
+// The envelope's sub-blocks must be blocks the metadata builder supports.
+eta_status_t check_sub_blocks(const eta_shape_t* s, const eta_params_t* p, bool paged) {
+  const int r = sub_blocks_of(p);
+  if (r == 1) return ETA_OK;
+  if (paged || s->block_size / r < 16) return ETA_ERR_UNSUPPORTED;
   return ETA_OK;
 }
 
@@ -188,12 +200,14 @@ eta_status_t do_screen(const eta_shape_t* s, const eta_params_t* p, const void* 
                        const float* tau, int64_t tau_stride, const eta_screen_out_t* out, const Workspace& w,
                        cudaStream_t st, const float* W = nullptr, const float* bias = nullptr,
                        float* tau_out = nullptr, const int32_t* seq_lens = nullptr) {
+  ETA_TRY(check_sub_blocks(s, p, false));
   ScreenCall c;
   c.seq_lens = seq_lens;
   c.shape = *s;
   c.z = p->z;
   c.offset_a = p->offset_a;
   c.n_local = p->n_local;
+  c.sub_blocks = sub_blocks_of(p);
   c.q = q;
   c.meta = meta;
   c.n = n;
@@ -520,6 +534,7 @@ ETA_API eta_status_t eta_decode_sparse_paged(const eta_shape_t* shape, const eta
                                              const eta_screen_out_t* extra, void* workspace, size_t ws_bytes,
                                              eta_stream_t stream) {
   ETA_TRY(check_common_decode(shape, params, q, k_pool, v_pool, max_tokens, out));
+  ETA_TRY(check_sub_blocks(shape, params, true));
   ETA_TRY(check_pages(pages));
   ETA_TRY(check_lens(seq_lens));
   ETA_TRY(check_screen_shape(shape));

@@ -81,6 +81,7 @@ struct ScreenCall {
   eta_shape_t shape;
   float z, offset_a;
   int n_local;
+  int sub_blocks;          // r: sub-blocks per block (1 = Eq. 5 on whole blocks)
   const void* q;
   eta_meta_t meta;
   int64_t n;               // tokens (all rows), or the upper bound of seq_lens

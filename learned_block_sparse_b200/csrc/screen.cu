@@ -41,12 +41,13 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
   screen_prologue<D, G, 32, true>(a, sm, b, kvh, kScreenWarps * 32);
 
   const RowBlocks rb = row_blocks(a, b);
-  const int nt = (rb.ns + 31) / 32;
+  const int units = rb.ns * a.r;  // screened metadata columns (sub-blocks)
+  const int nt = (units + 31) / 32;
   const int t0 = cr * tpc;
   const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
-  const float* mu = a.mu + static_cast<int64_t>(bh) * D * a.nb_cap;
-  const float* var = a.var + static_cast<int64_t>(bh) * D * a.nb_cap;
-  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
+  const float* mu = a.mu + static_cast<int64_t>(bh) * D * a.nb_cap_meta;
+  const float* var = a.var + static_cast<int64_t>(bh) * D * a.nb_cap_meta;
+  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap_meta;
 
   // Phase 1: score and decide every screened block of this CTA's tiles.
   for (int t4 = warp * kSub; t4 < my_tiles; t4 += kScreenWarps * kSub) {
@@ -54,9 +55,9 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
     bool valid[kSub];
 #pragma unroll
     for (int u = 0; u < kSub; ++u) {
-      const int blk = (t0 + t4 + u) * 32 + lane;
-      valid[u] = (t4 + u < my_tiles) && blk < rb.ns;
-      cb[u] = blk < rb.ns ? blk : rb.ns - 1;  // rb.ns >= 1 here (this warp has a tile)
+      const int unit = (t0 + t4 + u) * 32 + lane;
+      valid[u] = (t4 + u < my_tiles) && unit < units;
+      cb[u] = unit < units ? unit : units - 1;  // units >= 1 here (this warp has a tile)
     }
     float dg[kSub][G], vg[kSub][G];
 #pragma unroll
@@ -68,8 +69,8 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
       float m[kSub], v[kSub];
 #pragma unroll
       for (int u = 0; u < kSub; ++u) {
-        m[u] = __ldg(mu + static_cast<int64_t>(i) * a.nb_cap + cb[u]);
-        v[u] = __ldg(var + static_cast<int64_t>(i) * a.nb_cap + cb[u]);
+        m[u] = __ldg(mu + static_cast<int64_t>(i) * a.nb_cap_meta + cb[u]);
+        v[u] = __ldg(var + static_cast<int64_t>(i) * a.nb_cap_meta + cb[u]);
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -100,7 +101,7 @@ cudaError_t launch_screen_t(const ScreenCall& c, cudaStream_t st) {
   const int BH = s.batch * s.n_kv_heads;
   const int nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
   const int ns = max(0, nb - c.n_local);
-  const int nt = (ns + 31) / 32;
+  const int nt = (ns * c.sub_blocks + 31) / 32;
   // As many CTAs per cluster as there are tiles, up to kMaxCluster.
   const int cs = max(1, min(kMaxCluster, nt));
   const int tpc = max(1, (nt + cs - 1) / cs);

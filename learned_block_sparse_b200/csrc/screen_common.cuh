@@ -27,6 +27,10 @@ struct ScreenArgs {
   float* tau_out;
   float z, s, offset_a;
   int Hq, Hkv, nb, ns, nb_cap, tiles_per_cta;  // nb, ns: of the longest row (launch sizing)
+  // Sub-block envelope: r sub-blocks per block, metadata columns nb_cap * r.
+  // A screening lane handles one metadata column ("unit"): sub-block u of
+  // block u / r; r = 1 is Eq. 5 on whole blocks.
+  int r, nb_cap_meta;
   const int32_t* seq_lens;  // [B] per-row token counts, or null (every row has n)
   int64_t n;
   int bs, n_local;
@@ -149,21 +153,35 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
   __syncthreads();
 }
 
-// Eq. 5 for one block and every head of the group, given the fma-accumulated
-// D = sum q_i mu_i and V = sum q_i^2 var_i: writes the scores (if asked) and
-// returns the head mask of the admitted heads.
+// Eq. 5 for one metadata unit and every head of the group, given the
+// fma-accumulated D = sum q_i mu_i and V = sum q_i^2 var_i; with sub-blocks
+// (r > 1) the block's score is the largest over its r units, which sit in r
+// consecutive lanes (r divides 32, and the r units of a block are all valid or
+// all invalid); the first of them decides the block. Writes the scores (if
+// asked) and returns the head mask of the admitted heads. All 32 lanes call it.
 template <int D, int G>
 __device__ __forceinline__ uint32_t screen_decide(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
-                                                  int blk, bool valid, const float (&dg)[G], const float (&vg)[G],
+                                                  int unit, bool valid, const float (&dg)[G], const float (&vg)[G],
                                                   float M) {
-  uint32_t mask = 0;
+  float sc[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const float A = __fadd_rn(dg[g], __fmul_rn(a.z, __fsqrt_rn(vg[g])));
     const float C = __fmul_rn(sm.qn[g], M);
-    const float sc = __fmul_rn((A < C) ? A : C, a.s);
-    if (valid && !(sc < sm.taut[g])) mask |= 1u << g;
-    if (a.scores != nullptr && valid) a.scores[(static_cast<int64_t>(b) * a.Hq + kvh * G + g) * a.nb_cap + blk] = sc;
+    sc[g] = __fmul_rn((A < C) ? A : C, a.s);
+  }
+  if (a.r > 1) {
+    for (int o = 1; o < a.r; o <<= 1)
+#pragma unroll
+      for (int g = 0; g < G; ++g) sc[g] = fmaxf(sc[g], __shfl_xor_sync(kFull, sc[g], o));
+    valid = valid && (threadIdx.x & (a.r - 1)) == 0;
+  }
+  const int blk = unit / a.r;
+  uint32_t mask = 0;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    if (valid && !(sc[g] < sm.taut[g])) mask |= 1u << g;
+    if (a.scores != nullptr && valid) a.scores[(static_cast<int64_t>(b) * a.Hq + kvh * G + g) * a.nb_cap + blk] = sc[g];
   }
   return mask;
 }
@@ -215,7 +233,7 @@ __device__ __forceinline__ void screen_finish(const ScreenArgs& a, const ScreenS
 
   const uint32_t lt = lanemask_lt();
   for (int t = warp; t < my_tiles; t += nwarps) {
-    const int blk = (t0 + t) * 32 + lane;
+    const int blk = ((t0 + t) * 32 + lane) / a.r;  // a lane with a mask bit is its block's first unit
     const uint32_t mask = sm.mask[t * 32 + lane];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -291,6 +309,8 @@ inline ScreenArgs make_screen_args(const ScreenCall& c, int nb, int ns, int tpc)
   a.n_local = c.n_local;
   a.status = c.ws.status;
   a.nb_cap = static_cast<int>(s.capacity / s.block_size);
+  a.r = c.sub_blocks;
+  a.nb_cap_meta = a.nb_cap * c.sub_blocks;
   a.tiles_per_cta = tpc;
   a.ws_union = c.ws.union_list;
   a.ws_union_cnt = c.ws.union_cnt;

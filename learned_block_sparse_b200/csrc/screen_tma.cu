@@ -75,7 +75,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   static_assert((static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>) % 16 == 0, "ScreenSmem alignment");
   const ScreenSmem<D, G> sm(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>, tpc);
 
-  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap;
+  const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap_meta;
 
   if (tid == 0) {
     *s_abort = 0;
@@ -89,7 +89,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   grid_dependency_wait();  // inputs may come from the previous kernel on the stream
   allow_dependent_launch();
   const RowBlocks rb = row_blocks(a, b);
-  const int nt = (rb.ns + 31) / 32;
+  const int units = rb.ns * a.r;  // screened metadata columns (sub-blocks)
+  const int nt = (units + 31) / 32;
   const int t0 = cr * tpc;
   const int my_tiles = max(0, min(nt, t0 + tpc) - t0);
   __syncthreads();
@@ -144,9 +145,9 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
     bool tau_waited = !tau_later;
     for (int it = warp; it < my_tiles; it += CW) {
       const int st = it % NST;
-      const int blk = (t0 + it) * 32 + lane;
-      const bool valid = blk < rb.ns;
-      const float M = __ldg(mx + (valid ? blk : rb.ns - 1));  // rb.ns >= 1 here (this CTA has a tile)
+      const int unit = (t0 + it) * 32 + lane;
+      const bool valid = unit < units;
+      const float M = __ldg(mx + (valid ? unit : units - 1));  // units >= 1 here (this CTA has a tile)
       const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status);
       float dg[G], vg[G];
 #pragma unroll
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
         tau_ok = mbar_wait_bounded(s_tau, 0u, s_abort, status);
         tau_waited = true;
       }
-      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, blk, valid && tau_ok, dg, vg, M));
+      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, unit, valid && tau_ok, dg, vg, M));
     }
   }
   __syncthreads();
@@ -204,7 +205,8 @@ PFN_cuTensorMapEncodeTiled_v12000 meta_map_encoder() {
   return fn;
 }
 
-// [rows][nb_cap] fp32 view of mu or var, boxes of [d rows][32 blocks].
+// [rows][ncol] fp32 view of mu or var (ncol metadata columns: blocks, or
+// sub-blocks with the envelope), boxes of [d rows][32 columns].
 bool encode_meta_map(CUtensorMap* tm, const float* base, int64_t rows, int64_t nb_cap, int d) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = meta_map_encoder();
   if (enc == nullptr) return false;
@@ -222,10 +224,10 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   constexpr int CW = TmaScreenCfg<D>::kCW, NST = TmaScreenCfg<D>::kNST;
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
-  const int64_t nb_cap = s.capacity / s.block_size;
+  const int64_t ncol = s.capacity / s.block_size * c.sub_blocks;
   const int nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
   const int ns = max(0, nb - c.n_local);
-  const int nt = (ns + 31) / 32;
+  const int nt = (ns * c.sub_blocks + 31) / 32;
   // Clusters as large as keeps the launch within one wave of two thread blocks
   // per SM (at least 1, at most kMaxCluster, at most one tile per CTA).
   int cs = static_cast<int>((2 * static_cast<int64_t>(device_sm_count())) / BH);
@@ -238,7 +240,7 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   if (smem > static_cast<size_t>(device_max_smem_optin())) return cudaErrorNotSupported;
   CUtensorMap tmu, tvar;
   const int64_t rows = static_cast<int64_t>(BH) * D;
-  if (!encode_meta_map(&tmu, c.meta.mu, rows, nb_cap, D) || !encode_meta_map(&tvar, c.meta.var, rows, nb_cap, D))
+  if (!encode_meta_map(&tmu, c.meta.mu, rows, ncol, D) || !encode_meta_map(&tvar, c.meta.var, rows, ncol, D))
     return cudaErrorNotSupported;
   const ScreenArgs a = make_screen_args(c, nb, ns, tpc);
   static std::atomic<uint64_t> smem_done{0};
@@ -277,9 +279,9 @@ cudaError_t launch_tma_d(const ScreenCall& c, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_screen_tma(const ScreenCall& c, cudaStream_t st) {
-  const int64_t nb_cap = c.shape.capacity / c.shape.block_size;
+  const int64_t ncol = c.shape.capacity / c.shape.block_size * c.sub_blocks;
   // TMA wants 16-byte aligned rows and a 16-byte aligned base
-  if (nb_cap % 4 != 0 || (reinterpret_cast<uintptr_t>(c.meta.mu) & 15) != 0 ||
+  if (ncol % 4 != 0 || (reinterpret_cast<uintptr_t>(c.meta.mu) & 15) != 0 ||
       (reinterpret_cast<uintptr_t>(c.meta.var) & 15) != 0)
     return cudaErrorNotSupported;
   return c.shape.head_dim == 128 ? launch_tma_d<128>(c, st) : launch_tma_d<64>(c, st);

@@ -99,6 +99,8 @@ class Workload:
     @property
     def capacity(self) -> int:
         if self.cap is not None:
+            if self.cap < self.n:
+                raise ValueError(f"capacity {self.cap} below the token count {self.n}")
             return ((self.cap + self.bs - 1) // self.bs) * self.bs
         q = 4 * self.bs          # whole groups of 4 blocks: 16-byte aligned metadata rows
         return ((self.n + q - 1) // q) * q

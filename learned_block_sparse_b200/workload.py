@@ -18,7 +18,8 @@ from . import binding, synth
 
 class DeviceWorkload:
     def __init__(self, w: synth.Workload, device="cuda", n_splits: int = 0, offset_a: float = 0.0,
-                 keep_host: bool = False, stage_bytes: int = 1 << 30, gate: int = binding.GATE_SIGMOID):
+                 keep_host: bool = False, stage_bytes: int = 1 << 30, gate: int = binding.GATE_SIGMOID,
+                 sub_blocks: int = 1):
         self.w = w
         self.device = torch.device(device)
         self.q_host = synth.make_q(w)
@@ -46,7 +47,8 @@ class DeviceWorkload:
             del stage
         self.dec = binding.EtaDecoder(w.B, w.Hq, w.Hkv, w.d, w.bs, w.capacity, kv_dtype=w.torch_dtype,
                                       q_dtype=w.q_torch_dtype, beta=w.beta, z=w.z, offset_a=offset_a,
-                                      n_local=w.n_local, n_splits=n_splits, device=self.device, gate=gate)
+                                      n_local=w.n_local, n_splits=n_splits, device=self.device, gate=gate,
+                                      sub_blocks=sub_blocks)
         self.dec.build_meta(self.K, 0, w.n // w.bs)
         self.W = self.bias0 = None
         if w.tau_mode == "predictor":

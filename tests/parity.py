@@ -25,32 +25,40 @@ def pmap(fn, items):
     return list(_POOL.map(lambda a: fn(*a), items))
 
 
-def oracle_meta(w: synth.Workload, K_host: torch.Tensor, pairs: Optional[Iterable] = None):
-    """Oracle metadata for the given (b, kvh) pairs (default all): dict -> (mu, var, mx)."""
+def oracle_meta(w: synth.Workload, K_host: torch.Tensor, pairs: Optional[Iterable] = None, r: int = 1):
+    """Oracle metadata for the given (b, kvh) pairs (default all): dict -> (mu, var, mx);
+    with r > 1, of the sub-blocks of w.bs / r tokens (the sub-block envelope)."""
     Kraw = K_host
-    nf = w.n // w.bs
+    nf = (w.n // w.bs) * r
     pairs = list(pairs) if pairs is not None else [(b, h) for b in range(w.B) for h in range(w.Hkv)]
 
     def one(b, h):
-        return (b, h), oracle.slice_meta(Kraw[b, h], w.d, w.bs, nf)
+        return (b, h), oracle.slice_meta(Kraw[b, h], w.d, w.bs // r, nf)
     return dict(pmap(one, [(b, h) for (b, h) in pairs]))
 
 
-def oracle_scores(w, qf: np.ndarray, meta: dict, heads):
+def screen(qf, mu, var, mx, w, tau, offset_a=0.0, r=1):
+    """The oracle screen of one head: Eq. 5 on whole blocks, or the sub-block envelope."""
+    if r > 1:
+        return oracle.screen_head_env(qf, mu, var, mx, w.nb, r, w.n_local, w.z, tau, offset_a)
+    return oracle.screen_head(qf, mu, var, mx, w.nb, w.n_local, w.z, tau, offset_a)
+
+
+def oracle_scores(w, qf: np.ndarray, meta: dict, heads, r=1):
     def one(b, hq):
         mu, var, mx = meta[(b, hq // w.G)]
-        _, sc = oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, float("-inf"))
+        _, sc = screen(qf[b, hq], mu, var, mx, w, float("-inf"), r=r)
         return (b, hq), sc
     return dict(pmap(one, heads))
 
 
-def oracle_thresholds(w, q_host, meta, density, W=None, heads=None):
+def oracle_thresholds(w, q_host, meta, density, W=None, heads=None, r=1):
     """Thresholds for a target density, computed on the oracle side.
     const: per-head constant over the batch, returns (tau [Hq], stride 0, None).
     predictor: returns (tau [B][Hq], stride Hq, bias [Hq])."""
     qf = oracle.to_f32(q_host)
     all_heads = [(b, h) for b in range(w.B) for h in range(w.Hq)]
-    sc = oracle_scores(w, qf, meta, heads or all_heads)
+    sc = oracle_scores(w, qf, meta, heads or all_heads, r=r)
     if w.tau_mode == "const":
         tau = np.zeros((w.Hq,), np.float32)
         for h in range(w.Hq):
@@ -107,7 +115,7 @@ def run_gpu(dw, tau, stride, bias=None, dense=False):
 
 
 def oracle_step(w, q_host, K_host, V_host, meta, tau, stride, heads, dense=False, offset_a=0.0,
-                gate=oracle.GATE_SIGMOID):
+                gate=oracle.GATE_SIGMOID, r=1):
     qf = oracle.to_f32(q_host)
     tau_arr = np.asarray(tau, np.float32)
 
@@ -120,7 +128,7 @@ def oracle_step(w, q_host, K_host, V_host, meta, tau, stride, heads, dense=False
             lst, sc = np.arange(w.nb, dtype=np.int32), None
         else:
             mu, var, mx = meta[(b, kvh)]
-            lst, sc = oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, tau_of(b, hq), offset_a)
+            lst, sc = screen(qf[b, hq], mu, var, mx, w, tau_of(b, hq), offset_a, r)
         t_gate = float("-inf") if (dense and tau is None) else tau_of(b, hq)
         o = oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, w.n, qf[b, hq], lst, t_gate, w.beta, gate)
         return (b, hq), (lst, sc, o)

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_abi_version_and_status_strings():
     from learned_block_sparse_b200 import binding
-    assert binding.lib.eta_abi_version() == 2
+    assert binding.lib.eta_abi_version() == 3
     assert binding.status_string(0) == "ok"
     assert "workspace" in binding.status_string(3)
     assert binding.status_string(99) == "unknown status"
@@ -91,7 +91,8 @@ def test_argument_validation_before_launch():
                                a16, 64, None) == 3
     # params
     for bad_p in (binding.make_params(beta=0.0), binding.make_params(n_local=0), binding.make_params(n_splits=-1),
-                  binding.make_params(z=float("nan")), binding.make_params(gate=2)):
+                  binding.make_params(z=float("nan")), binding.make_params(gate=2),
+                  binding.make_params(sub_blocks=3), binding.make_params(sub_blocks=-1)):
         assert L.eta_decode_dense(ctypes.byref(s), ctypes.byref(bad_p), a16, a16, a16, 100, None, 0, a16, a16,
                                   1 << 30, None) == 1
     # per-row lengths: the length array is required; max_tokens bounded by the capacity
@@ -101,6 +102,17 @@ def test_argument_validation_before_launch():
                                      a16, a16, 1 << 30, None) == 1
     assert L.eta_decode_sparse_ragged(ctypes.byref(s), ctypes.byref(p), a16, a16, a16, meta, a16, 100, None, 0,
                                       None, None, None, a16, None, a16, 1 << 30, None) == 1   # no thresholds
+    # sub-block envelope: sub-blocks of fewer than 16 tokens, and paged stores, are not supported
+    for bs, r in ((32, 4), (16, 2)):
+        s2 = _shape(block_size=bs)
+        p2 = binding.make_params(sub_blocks=r)
+        assert L.eta_screen(ctypes.byref(s2), ctypes.byref(p2), a16, meta, 100, a16, 0, None, a16, 1 << 30,
+                            None) == 2, (bs, r)
+    assert L.eta_decode_workspace_bytes(ctypes.byref(s), ctypes.byref(binding.make_params(sub_blocks=2))) > 0
+    pages = binding.Pages(1 << 20, 64)
+    p2 = binding.make_params(sub_blocks=2)
+    assert L.eta_decode_sparse_paged(ctypes.byref(s), ctypes.byref(p2), a16, a16, a16, pages, meta, a16, 100, a16,
+                                     0, None, None, None, a16, None, a16, 1 << 30, None) == 2
     # metadata block range
     assert L.eta_build_block_meta(ctypes.byref(s), a16, -1, 3, meta, None) == 1
     assert L.eta_build_block_meta(ctypes.byref(s), a16, 0, 33, meta, None) == 1

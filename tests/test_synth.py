@@ -91,3 +91,10 @@ def test_tau_for_density():
     assert (s >= t).sum() == 38
     assert synth.tau_for_density(s, 1.0) == float("-inf")
     assert (s >= synth.tau_for_density(s, 0.001)).sum() == 1
+
+
+def test_capacity_below_the_token_count_is_rejected():
+    w = synth.Workload("c", "bf16", 1, 2, 2, 64, 1000, 16, z=1.0, tau_mode="const", densities=(0.5,), seed=1,
+                       cap=512)
+    with pytest.raises(ValueError):
+        _ = w.capacity
