@@ -52,6 +52,8 @@ def parse_args():
     p.add_argument("--density", type=float, default=None,
                    help="target admitted fraction (default: the middle density of the workload)")
     p.add_argument("--n-splits", type=int, default=0)
+    p.add_argument("--sub-blocks", type=int, default=1, choices=[1, 2, 4, 8],
+                   help="sub-block envelope: metadata per sub-block of b/r tokens, a block scored by its best one")
     p.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     p.add_argument("--no-dense", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -194,7 +196,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ byte models
-def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
+def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int, r: int = 1):
     """Algorithmic bytes of one step from the admitted counts.
     union_cnt [B][Hkv]; the last block of each list is partial when n % b != 0."""
     eb = {"f32": 4, "bf16": 2, "fp8": 1}[w.dtype]
@@ -221,7 +223,7 @@ def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
     partials = partial_rows * w.G * (w.d + 2) * 4
     out = w.B * w.Hq * w.d * 4
     decode = kv + lists_read + q + partials + out
-    meta = bh * w.n_screened * (2 * w.d + 1) * 4
+    meta = bh * w.n_screened * r * (2 * w.d + 1) * 4   # r metadata columns per block with the envelope
     W = (w.Hq * w.d * w.Hq * 4 + w.Hq * 4) if w.tau_mode == "predictor" else 0
     step_read = kv + meta + lists_read + q * 2 + W
     dense_kv = 2 * row * bh * w.n
@@ -232,21 +234,29 @@ def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int):
 
 
 # -------------------------------------------------------------- CPU oracle
-def oracle_setup(w, dw_host, groups):
+def oracle_screen(w, qf_h, meta, t, r):
+    """The oracle screen of one head: Eq. 5 on whole blocks, or the sub-block envelope."""
+    import oracle
+    mu, var, mx = meta
+    if r > 1:
+        return oracle.screen_head_env(qf_h, mu, var, mx, w.nb, r, w.n_local, w.z, t)
+    return oracle.screen_head(qf_h, mu, var, mx, w.nb, w.n_local, w.z, t)
+
+
+def oracle_setup(w, dw_host, groups, r=1):
     """Oracle-side metadata and thresholds for the sampled (b, kv head) groups."""
     import oracle
     from learned_block_sparse_b200 import synth
     q_host, K_host, V_host = dw_host
-    nf = w.n // w.bs
+    nf = (w.n // w.bs) * r
     pool = cf.ThreadPoolExecutor(max_workers=os.cpu_count() or 1)
-    metas = dict(zip(groups, pool.map(lambda g: oracle.slice_meta(K_host[g[0], g[1]], w.d, w.bs, nf), groups)))
+    metas = dict(zip(groups, pool.map(lambda g: oracle.slice_meta(K_host[g[0], g[1]], w.d, w.bs // r, nf), groups)))
     qf = oracle.to_f32(q_host)
     heads = [(b, kvh * w.G + g) for (b, kvh) in groups for g in range(w.G)]
 
     def sc(bh):
         b, hq = bh
-        mu, var, mx = metas[(b, hq // w.G)]
-        return oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, float("-inf"))[1]
+        return oracle_screen(w, qf[b, hq], metas[(b, hq // w.G)], float("-inf"), r)[1]
     scores = dict(zip(heads, pool.map(sc, heads)))
     return metas, qf, heads, scores, pool
 
@@ -268,7 +278,7 @@ def oracle_thresholds(w, q_host, W, scores, density):
     return ("predictor", None, bias)
 
 
-def oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool):
+def oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool, r=1):
     """One oracle decode step over the sampled heads: predictor, screen, gated attention."""
     import oracle
     kind, tau_c, bias = thr
@@ -278,8 +288,7 @@ def oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool):
         b, hq = bh
         kvh = hq // w.G
         t = float(tau[b, hq]) if tau is not None else float(tau_c[hq])
-        mu, var, mx = metas[(b, kvh)]
-        lst, _ = oracle.screen_head(qf[b, hq], mu, var, mx, w.nb, w.n_local, w.z, t)
+        lst, _ = oracle_screen(w, qf[b, hq], metas[(b, kvh)], t, r)
         return oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, w.n, qf[b, hq], lst, t, w.beta)
     return list(pool.map(one, heads))
 
@@ -300,13 +309,13 @@ def run_reference(args):
     groups = sorted(groups_all[i] for i in rng.choice(len(groups_all), n_groups, replace=False))
     q_host, K_host, V_host = host_slices(w, groups)
     W = synth.make_predictor(w)[0].numpy() if w.tau_mode == "predictor" else None
-    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups)
+    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups, args.sub_blocks)
     thr = oracle_thresholds(w, q_host, W, scores, args.density)
     for _ in range(args.warmup):
-        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool, args.sub_blocks)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool, args.sub_blocks)
     dt = (time.perf_counter() - t0) / args.steps
     value = len(heads) / dt
     cores = pool._max_workers
@@ -314,7 +323,8 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": w.name, "density": args.density, "batch": w.B, "seq_len": w.n},
+            "config": {"workload": w.name, "density": args.density, "batch": w.B, "seq_len": w.n,
+                       **({"sub_blocks": args.sub_blocks} if args.sub_blocks > 1 else {})},
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
                              "sample": f"{len(heads)} decode queries ({n_groups} (batch, kv head) groups) of "
                                        f"the workload per step"},
@@ -346,7 +356,7 @@ def run_eta(args):
     if args.batch:
         w = w.replace(B=args.batch)
     dev = torch.device("cuda", torch.cuda.current_device())
-    dw = DeviceWorkload(w, device=dev, n_splits=args.n_splits)
+    dw = DeviceWorkload(w, device=dev, n_splits=args.n_splits, sub_blocks=args.sub_blocks)
     dec = dw.dec
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -422,7 +432,7 @@ def run_eta(args):
             binding.screen(dec.shape, dec.params, dw.q, dec.meta, w.n, tau, stride, dec.ws, union_cnt=ucnt,
                            active_cnt=hcnt)
         torch.cuda.synchronize()
-        bm = byte_model(w, ucnt.cpu().numpy(), hcnt.cpu().numpy(), S)
+        bm = byte_model(w, ucnt.cpu().numpy(), hcnt.cpu().numpy(), S, args.sub_blocks)
         st = dec.device_status()
         if st != 0:
             raise RuntimeError(f"device status {st} after timed steps")
@@ -489,6 +499,7 @@ def run_eta(args):
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller normals, shaped like the pages' decode workloads)",
         "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
                    "seq_len": w.n, "block": w.bs, "tau": w.tau_mode, "density_target": args.density,
+                   **({"sub_blocks": args.sub_blocks} if args.sub_blocks > 1 else {}),
                    "l2": ("flushed before every timed step: 512 MiB write" +
                           (", then a 512 MiB read (no dirty lines left)" if args.l2_flush == "write+read" else "")), "parallelism": f"replicas x{world}"},
         "effective_hbm_gbs": bm["step_read"] / (ms * 1e-3) / 1e9,
@@ -561,13 +572,13 @@ def cpu_baseline(w, args, dw):
     groups = sorted(groups_all[i] for i in rng.choice(len(groups_all), n, replace=False))
     q_host, K_host, V_host = host_slices(w, groups)
     W = synth.make_predictor(w)[0].numpy() if w.tau_mode == "predictor" else None
-    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups)
+    metas, qf, heads, scores, pool = oracle_setup(w, (q_host, K_host, V_host), groups, args.sub_blocks)
     thr = oracle_thresholds(w, q_host, W, scores, args.density)
     # repeat the step until about 5 s have passed (bounded at 200 steps)
     t0 = time.perf_counter()
     reps = 0
     while reps < 200:
-        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool)
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool, args.sub_blocks)
         reps += 1
         if time.perf_counter() - t0 >= 5.0:
             break
