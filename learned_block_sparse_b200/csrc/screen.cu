@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kScreenWarps * 32, 4) screen_kernel(const Scre
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float qi = sm.q[g * D + i], qqi = sm.qq[g * D + i];
+        const float qi = sm.q[i * G + g], qqi = sm.qq[i * G + g];
 #pragma unroll
         for (int u = 0; u < kSub; ++u) {
           dg[u][g] = __fmaf_rn(qi, m[u], dg[u][g]);

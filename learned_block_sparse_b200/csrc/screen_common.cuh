@@ -60,8 +60,8 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 // Shared-memory carve-up common to both kernels (offsets from `base`).
 template <int D, int G>
 struct ScreenSmem {
-  float* q;      // [G][D]
-  float* qq;     // [G][D] fl(q_i * q_i)
+  float* q;      // [D][G] (head-minor: the G heads of a coordinate are adjacent)
+  float* qq;     // [D][G] fl(q_i * q_i)
   float* qn;     // [G] fl(sqrt(sum q_i^2))
   float* taut;   // [G] tau - a
   int* tot;      // [G+1] this CTA's admitted counts
@@ -130,8 +130,8 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
   for (int i = tid; i < G * D; i += nthreads) {
     const int g = i / D, e = i % D;
     const float x = load_elem(a.q, a.q_dtype, (static_cast<int64_t>(b) * a.Hq + kvh * G + g) * D + e);
-    sm.q[i] = x;
-    sm.qq[i] = __fmul_rn(x, x);
+    sm.q[e * G + g] = x;
+    sm.qq[e * G + g] = __fmul_rn(x, x);
   }
   if (a.W == nullptr) {
     if (tid < G) sm.taut[tid] = __fsub_rn(a.tau[b * a.tau_stride + kvh * G + tid], a.offset_a);
@@ -144,7 +144,7 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
     for (int e0 = 0; e0 < D; e0 += 16) {
       float x[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) x[c] = sm.q[tid * D + e0 + c];
+      for (int c = 0; c < 16; ++c) x[c] = sm.q[(e0 + c) * G + tid];
 #pragma unroll
       for (int c = 0; c < 16; ++c) qn = __fmaf_rn(x[c], x[c], qn);
     }

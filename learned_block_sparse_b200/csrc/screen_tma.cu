@@ -47,6 +47,20 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
       : "memory");
 }
 
+// Packed fp32 pairs: fma.rn.f32x2 performs two independent IEEE fused
+// multiply-adds, each rounding as __fmaf_rn does.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2)
     screen_tma_kernel(const ScreenArgs a, int32_t* status, const __grid_constant__ CUtensorMap tmu,
@@ -155,27 +169,49 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
       if (ok) {
         const float* mu_s = s_stage + static_cast<size_t>(st) * 2 * D * 32;
         const float* var_s = mu_s + D * 32;
+        if constexpr (G == 1) {
 #pragma unroll 2
-        for (int i0 = 0; i0 < D; i0 += 4) {
-          float m[4], v[4];
+          for (int i0 = 0; i0 < D; i0 += 4) {
+            // four coordinates of q and q*q per shared load; multiply-adds in coordinate order
+            const float4 qv = *reinterpret_cast<const float4*>(sm.q + i0);
+            const float4 qqv = *reinterpret_cast<const float4*>(sm.qq + i0);
+            const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, qqa[4] = {qqv.x, qqv.y, qqv.z, qqv.w};
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            m[c] = mu_s[(i0 + c) * 32 + lane];
-            v[c] = var_s[(i0 + c) * 32 + lane];
+            for (int c = 0; c < 4; ++c) {
+              dg[0] = __fmaf_rn(qa[c], mu_s[(i0 + c) * 32 + lane], dg[0]);
+              vg[0] = __fmaf_rn(qqa[c], var_s[(i0 + c) * 32 + lane], vg[0]);
+            }
+          }
+        } else {
+          // heads 2p and 2p+1 share a packed multiply-add per coordinate: the
+          // [D][G] query rows give both of a coordinate's factors in one load
+          const uint64_t* q2 = reinterpret_cast<const uint64_t*>(sm.q);
+          const uint64_t* qq2 = reinterpret_cast<const uint64_t*>(sm.qq);
+          uint64_t d2[G / 2], v2[G / 2];
+#pragma unroll
+          for (int p = 0; p < G / 2; ++p) d2[p] = v2[p] = 0ull;  // +0.0f in both halves
+#pragma unroll 2
+          for (int i0 = 0; i0 < D; i0 += 4) {
+            float m[4], v[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              m[c] = mu_s[(i0 + c) * 32 + lane];
+              v[c] = var_s[(i0 + c) * 32 + lane];
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint64_t mm = pack2(m[c], m[c]), vv = pack2(v[c], v[c]);
+#pragma unroll
+              for (int p = 0; p < G / 2; ++p) {
+                fma2(d2[p], q2[(i0 + c) * (G / 2) + p], mm);
+                fma2(v2[p], qq2[(i0 + c) * (G / 2) + p], vv);
+              }
+            }
           }
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            // four coordinates of q and q*q per shared load; multiply-adds in coordinate order
-            const float4 qv = *reinterpret_cast<const float4*>(sm.q + g * D + i0);
-            const float4 qqv = *reinterpret_cast<const float4*>(sm.qq + g * D + i0);
-            dg[g] = __fmaf_rn(qv.x, m[0], dg[g]);
-            dg[g] = __fmaf_rn(qv.y, m[1], dg[g]);
-            dg[g] = __fmaf_rn(qv.z, m[2], dg[g]);
-            dg[g] = __fmaf_rn(qv.w, m[3], dg[g]);
-            vg[g] = __fmaf_rn(qqv.x, v[0], vg[g]);
-            vg[g] = __fmaf_rn(qqv.y, v[1], vg[g]);
-            vg[g] = __fmaf_rn(qqv.z, v[2], vg[g]);
-            vg[g] = __fmaf_rn(qqv.w, v[3], vg[g]);
+          for (int p = 0; p < G / 2; ++p) {
+            unpack2(d2[p], dg[2 * p], dg[2 * p + 1]);
+            unpack2(v2[p], vg[2 * p], vg[2 * p + 1]);
           }
         }
       }
