@@ -57,7 +57,7 @@ typedef struct CUstream_st* eta_stream_t; /* same type as cudaStream_t */
 typedef enum {
   ETA_OK = 0,
   ETA_ERR_INVALID_ARG = 1,    /* a null pointer, bad size, misaligned pointer */
-  ETA_ERR_UNSUPPORTED = 2,    /* a shape this build has no kernel for */
+  ETA_ERR_UNSUPPORTED = 2,    /* a shape the library has no kernel for */
   ETA_ERR_WORKSPACE = 3,      /* workspace null, misaligned or too small */
   ETA_ERR_CUDA = 4,           /* a CUDA runtime call or launch failed */
   ETA_ERR_DEVICE_TIMEOUT = 5  /* a device-side wait exceeded its limit */
