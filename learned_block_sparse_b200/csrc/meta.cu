@@ -12,93 +12,127 @@ namespace eta {
 
 namespace {
 
-constexpr int kMetaThreads = 128;
-constexpr int kMetaTile = 32;  // blocks per thread block (one coalesced 128-byte row per coordinate)
+constexpr int kMetaWarps = 8;  // blocks in work per thread block: one warp each
 
+// Coordinate p of a 32-bit word of the store (4 / elt coordinates per word),
+// widened exactly to fp32.
+template <typename KV>
+__device__ __forceinline__ float word_elem(uint32_t w, int p);
+template <>
+__device__ __forceinline__ float word_elem<float>(uint32_t w, int) {
+  return __uint_as_float(w);
+}
+template <>
+__device__ __forceinline__ float word_elem<Bf16Raw>(uint32_t w, int p) {
+  return p == 0 ? bf16_lo(w) : bf16_hi(w);
+}
+template <>
+__device__ __forceinline__ float word_elem<Fp8Raw>(uint32_t w, int p) {
+  return e4m3_to_float((w >> (8 * p)) & 0xffu);
+}
+
+// One warp per block. Row norms: lane r takes rows r, r+32, ... and folds
+// x_i^2 in increasing i (each row read as 16-byte chunks); the block's largest
+// norm by a max butterfly. Centroid and variance: lane l takes the words l,
+// l+32, ... of every row (elt-wide coordinates packed in 32 bits) and folds the
+// rows in increasing order, a first pass for the sum, a second for the squared
+// deviations from the rounded mean (the block was just read: the second and the
+// column reads come from the L1/L2 caches). Every sum keeps the order of a
+// sequential loop, so the metadata does not depend on the launch shape.
 template <typename KV, int D>
-__global__ void __launch_bounds__(kMetaThreads) meta_kernel(const KV* __restrict__ k, const KvLayout L,
-                                                            int64_t nb_cap, int64_t blk_begin, int64_t blk_end,
-                                                            float* __restrict__ mu, float* __restrict__ var,
-                                                            float* __restrict__ maxn) {
-  extern __shared__ __align__(16) float sm[];
+__global__ void __launch_bounds__(kMetaWarps * 32) meta_kernel(const KV* __restrict__ k, const KvLayout L,
+                                                               int64_t nb_cap, int64_t blk_begin, int64_t blk_end,
+                                                               float* __restrict__ mu, float* __restrict__ var,
+                                                               float* __restrict__ maxn) {
+  constexpr int EB = KvTraits<KV>::kBytes;
+  constexpr int P = 4 / EB;          // coordinates per 32-bit word
+  constexpr int WPR = D / P;         // words per row
+  constexpr int C16 = D * EB / 16;   // 16-byte chunks per row
+  static_assert(WPR % 32 == 0, "words per row: a multiple of the warp");
+  constexpr int WL = WPR / 32;       // words of a row per lane
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
   const int bs = L.bs;
-  float* kb = sm;                             // [bs][D+1] widened keys of one block
-  float* s_mu = kb + bs * (D + 1);            // [D][kMetaTile]
-  float* s_var = s_mu + D * kMetaTile;        // [D][kMetaTile]
-  float* s_nrm = s_var + D * kMetaTile;       // [bs] squared row norms
-  float* s_mx = s_nrm + 128;                  // [kMetaTile]
-  const int tid = threadIdx.x;
-  const int64_t bh = blockIdx.x;
-  const int64_t j0 = blk_begin + static_cast<int64_t>(blockIdx.y) * kMetaTile;
-  const int jn = static_cast<int>((blk_end - j0 < kMetaTile ? blk_end - j0 : int64_t{kMetaTile}));
-  const int dt = KvTraits<KV>::kDtype;
   const float rows = static_cast<float>(bs);
-
-  for (int jj = 0; jj < jn; ++jj) {
-    const int64_t tok0 = kv_block_row(L, static_cast<int>(bh), static_cast<int>(j0 + jj));
-    if (tok0 < 0) {  // page outside the pool: nothing is read or written for this block (s_mx < 0)
-      if (tid < D) s_mu[tid * kMetaTile + jj] = s_var[tid * kMetaTile + jj] = 0.0f;
-      if (tid == 0) s_mx[jj] = -1.0f;
-      __syncthreads();
-      continue;
-    }
-    for (int idx = tid; idx < bs * D; idx += kMetaThreads) {
-      const int r = idx / D, i = idx % D;
-      kb[r * (D + 1) + i] = load_elem(k, dt, (tok0 + r) * D + i);
-    }
-    __syncthreads();
-    if (tid < D) {
-      float t = 0.0f;
-      for (int r = 0; r < bs; ++r) t = __fadd_rn(t, kb[r * (D + 1) + tid]);
-      const float m = __fdiv_rn(t, rows);
-      float v = 0.0f;
-      for (int r = 0; r < bs; ++r) {
-        const float e = __fsub_rn(kb[r * (D + 1) + tid], m);
-        v = __fmaf_rn(e, e, v);
-      }
-      s_mu[tid * kMetaTile + jj] = m;
-      s_var[tid * kMetaTile + jj] = __fdiv_rn(v, rows);
-    }
-    if (tid < bs) {
+  for (int64_t j = blk_begin + static_cast<int64_t>(blockIdx.y) * kMetaWarps + warp; j < blk_end;
+       j += static_cast<int64_t>(gridDim.y) * kMetaWarps) {
+    const int tok0 = kv_block_row(L, bh, static_cast<int>(j));
+    if (tok0 < 0) continue;  // page outside the pool: nothing is read or written for this block
+    const unsigned char* base = reinterpret_cast<const unsigned char*>(k) + static_cast<int64_t>(tok0) * D * EB;
+    float best = 0.0f;
+    for (int r = lane; r < bs; r += 32) {
+      const uint4* row = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(r) * D * EB);
       float nr = 0.0f;
-      for (int i = 0; i < D; ++i) {
-        const float x = kb[tid * (D + 1) + i];
-        nr = __fmaf_rn(x, x, nr);
+#pragma unroll
+      for (int c = 0; c < C16; ++c) {
+        const uint4 u = __ldg(row + c);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int p = 0; p < P; ++p) {
+            const float x = word_elem<KV>(w[q], p);
+            nr = __fmaf_rn(x, x, nr);
+          }
       }
-      s_nrm[tid] = nr;
+      best = fmaxf(best, nr);
     }
-    __syncthreads();
-    if (tid < 32) {
-      float best = 0.0f;
-      for (int r = tid; r < bs; r += 32) best = fmaxf(best, s_nrm[r]);
-      for (int o = 16; o >= 1; o >>= 1) best = fmaxf(best, __shfl_xor_sync(kFull, best, o));
-      if (tid == 0) s_mx[jj] = __fsqrt_rn(best);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) best = fmaxf(best, __shfl_xor_sync(kFull, best, o));
+    const uint32_t* words = reinterpret_cast<const uint32_t*>(base);
+    float t[WL][P];
+#pragma unroll
+    for (int c = 0; c < WL; ++c)
+#pragma unroll
+      for (int p = 0; p < P; ++p) t[c][p] = 0.0f;
+    for (int r = 0; r < bs; ++r) {
+#pragma unroll
+      for (int c = 0; c < WL; ++c) {
+        const uint32_t w = __ldg(words + static_cast<int64_t>(r) * WPR + lane + 32 * c);
+#pragma unroll
+        for (int p = 0; p < P; ++p) t[c][p] = __fadd_rn(t[c][p], word_elem<KV>(w, p));
+      }
     }
-    __syncthreads();
+    float v[WL][P];
+#pragma unroll
+    for (int c = 0; c < WL; ++c)
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+        t[c][p] = __fdiv_rn(t[c][p], rows);  // the mean
+        v[c][p] = 0.0f;
+      }
+    for (int r = 0; r < bs; ++r) {
+#pragma unroll
+      for (int c = 0; c < WL; ++c) {
+        const uint32_t w = __ldg(words + static_cast<int64_t>(r) * WPR + lane + 32 * c);
+#pragma unroll
+        for (int p = 0; p < P; ++p) {
+          const float e = __fsub_rn(word_elem<KV>(w, p), t[c][p]);
+          v[c][p] = __fmaf_rn(e, e, v[c][p]);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < WL; ++c)
+#pragma unroll
+      for (int p = 0; p < P; ++p) {
+        const int i = (lane + 32 * c) * P + p;
+        const int64_t o = (static_cast<int64_t>(bh) * D + i) * nb_cap + j;
+        mu[o] = t[c][p];
+        var[o] = __fdiv_rn(v[c][p], rows);
+      }
+    if (lane == 0) maxn[static_cast<int64_t>(bh) * nb_cap + j] = __fsqrt_rn(best);
   }
-  __syncthreads();
-  for (int idx = tid; idx < D * kMetaTile; idx += kMetaThreads) {
-    const int i = idx / kMetaTile, jj = idx % kMetaTile;
-    if (jj < jn && s_mx[jj] >= 0.0f) {
-      const int64_t o = (bh * D + i) * nb_cap + j0 + jj;
-      mu[o] = s_mu[idx];
-      var[o] = s_var[idx];
-    }
-  }
-  if (tid < jn && s_mx[tid] >= 0.0f) maxn[bh * nb_cap + j0 + tid] = s_mx[tid];
 }
 
 template <typename KV, int D>
 cudaError_t launch_meta_t(const eta_shape_t& s, const void* k, int64_t b0, int64_t b1, const eta_meta_t& m,
                           cudaStream_t st, const int32_t* table, int num_pages) {
   const int bs = s.block_size;
-  const size_t smem = (static_cast<size_t>(bs) * (D + 1) + 2 * D * kMetaTile + 128 + kMetaTile) * sizeof(float);
-  static std::atomic<uint64_t> smem_done{0};
-  cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(meta_kernel<KV, D>));
-  if (e != cudaSuccess) return e;
   const int64_t nb_cap = s.capacity / bs;
+  const int64_t groups = (b1 - b0 + kMetaWarps - 1) / kMetaWarps;
   dim3 grid(static_cast<unsigned>(static_cast<int64_t>(s.batch) * s.n_kv_heads),
-            static_cast<unsigned>((b1 - b0 + kMetaTile - 1) / kMetaTile));
+            static_cast<unsigned>(groups < 65535 ? groups : 65535));
   KvLayout L;
   L.block_table = table;
   L.max_blocks = static_cast<int>(nb_cap);
@@ -106,8 +140,8 @@ cudaError_t launch_meta_t(const eta_shape_t& s, const void* k, int64_t b0, int64
   L.Hkv = s.n_kv_heads;
   L.bs = bs;
   L.cap = s.capacity;
-  meta_kernel<KV, D><<<grid, kMetaThreads, smem, st>>>(static_cast<const KV*>(k), L, nb_cap, b0, b1, m.mu, m.var,
-                                                       m.maxnorm);
+  meta_kernel<KV, D><<<grid, kMetaWarps * 32, 0, st>>>(static_cast<const KV*>(k), L, nb_cap, b0, b1, m.mu, m.var,
+                                                        m.maxnorm);
   return cudaGetLastError();
 }
 
