@@ -583,10 +583,23 @@ def cpu_baseline(w, args, dw):
         if time.perf_counter() - t0 >= 5.0:
             break
     dt = time.perf_counter() - t0
+    # the same step on one thread, for the first group's heads (about 2 s)
+    one = cf.ThreadPoolExecutor(max_workers=1)
+    heads1 = heads[:w.G]
+    t1 = time.perf_counter()
+    reps1 = 0
+    while reps1 < 200:
+        oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads1, one, args.sub_blocks)
+        reps1 += 1
+        if time.perf_counter() - t1 >= 2.0:
+            break
+    dt1 = time.perf_counter() - t1
+    one.shutdown()
     return {"value": reps * len(heads) / dt, "unit": "queries/s", "cores": pool._max_workers, "kind": "oracle",
             "sample": f"{len(heads)} decode queries ({n} of {len(groups_all)} (batch, kv head) groups) per step, "
                       f"{reps} steps: predictor + screen + gated attention in C (fp32 decisions, fp64 attention)",
-            "seconds": dt}
+            "seconds": dt, "value_1_thread": reps1 * len(heads1) / dt1,
+            "sample_1_thread": f"{len(heads1)} decode queries (one group) per step, {reps1} steps"}
 
 
 def main():
