@@ -130,3 +130,33 @@ def test_workspace_size_grows_with_splits_and_capacity():
     b = binding.workspace_bytes(s, binding.make_params(n_splits=8))
     c = binding.workspace_bytes(_shape(capacity=4096), binding.make_params(n_splits=8))
     assert a < b < c and a % 256 == 0
+
+
+def test_binding_structs_match_the_header(tmp_path):
+    """The ctypes mirrors of eta_shape_t, eta_params_t, eta_meta_t, eta_pages_t and
+    eta_screen_out_t have the header's sizes and field offsets (a C probe compiled
+    against include/eta.h)."""
+    from learned_block_sparse_b200 import binding
+    structs = {"eta_shape_t": binding.Shape, "eta_params_t": binding.Params, "eta_meta_t": binding.Meta,
+               "eta_pages_t": binding.Pages, "eta_screen_out_t": binding.ScreenOut}
+    lines = ['#include <stddef.h>', '#include <stdio.h>', '#include "eta.h"', 'int main(void) {']
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines += ['  return 0;', '}']
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", "/usr/local/cuda/include", str(src), "-o",
+                    str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line:
+            c, f, v = line.split()
+            got[(c, f)] = int(v)
+    for cname, py in structs.items():
+        assert got[(cname, "size")] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[(cname, fname)] == getattr(py, fname).offset, (cname, fname)
