@@ -72,10 +72,29 @@ def parse_args():
 
 
 # ----------------------------------------------------------------- plumbing
+def relaunch_command(argv, n: int, port: int):
+    """The torch.distributed.run command that starts n ranks of this script
+    with the same arguments (one process per GPU, rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def launch_ranks(args) -> int:
+    """`bench.py --gpus N` (N > 1) started as a plain process: start the N ranks
+    and return their launcher's exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    return subprocess.call(relaunch_command(sys.argv[1:], args.gpus, port))
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
     if world > 1:
         import torch.distributed as dist
         torch.cuda.set_device(local)
@@ -144,55 +163,106 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled DURING the timed region.
 
-    def __init__(self, device_index: int):
+    A thread polls NVML about once a millisecond from start() to stop(), so
+    that a timed region of a few tens of milliseconds still gets tens of
+    samples; when NVML is not importable it falls back to nvidia-smi's
+    20 ms loop. The device is found by its UUID (CUDA and NVML may number
+    GPUs differently)."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.dev = device_index
+        self.period = period_s
+        self.samples = []          # (sm_mhz, max_mhz, reasons bitmask)
+        self.thread = None
         self.proc = None
         self.path = None
+        self.source = None
+        self._stop = False
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
+        try:
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            read = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+
+            def loop():
+                while not self._stop:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx, int(read(h))))
+                    time.sleep(self.period)
+            import threading
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.source = "nvml, ~1 ms polling"
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi -lms 20"
         except Exception:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    def _smi_samples(self):
+        names = [nm for nm, _ in self.REASONS[:4]]
+        bits = dict(self.REASONS)
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
+                    sm, mx = float(parts[1]), float(parts[2])
                 except ValueError:
                     continue
+                mask = 0
                 for nm, val in zip(names, parts[5:9]):
                     if val.lower() == "active":
-                        reasons.add(nm)
+                        mask |= bits[nm]
+                self.samples.append((sm, mx, mask))
         os.unlink(self.path)
-        if not sm:
+
+    def stop(self):
+        if self.thread is not None:
+            self._stop = True
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            time.sleep(0.05)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self._smi_samples()
+        else:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return None
+        reasons = sorted({nm for (_, _, m) in self.samples for nm, bit in self.REASONS if m & bit})
+        sm = [x[0] for x in self.samples]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "sm_mhz_min": min(sm), "reasons": reasons, "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------------ byte models
@@ -294,9 +364,17 @@ def oracle_step(w, q_host, K_host, V_host, W, thr, metas, qf, heads, pool, r=1):
 
 
 def run_reference(args):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only; the other ranks join
+    the CPU process group and exit without work)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {world} ranks")
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+        dist.barrier()
+        dist.destroy_process_group()
     if rank != 0:
         return
     from learned_block_sparse_b200 import synth
@@ -413,15 +491,16 @@ def run_eta(args):
         torch.cuda.synchronize()
         barrier(world)
         clocks = clk.stop() if clk else None
-        tot = sum(e[0].elapsed_time(e[2]) for e in evs) / args.steps
+        per_step = [e[0].elapsed_time(e[2]) for e in evs]
+        tot = statistics.median(per_step)
         # the same steps with an event between the launches, for the phase split
         pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
         for i in range(args.steps):
             flush.zero_()
             step_phases(tau, stride, bias, pevs[i])
         torch.cuda.synchronize()
-        scr = sum(e[0].elapsed_time(e[1]) for e in pevs) / args.steps
-        dec_t = sum(e[1].elapsed_time(e[2]) for e in pevs) / args.steps
+        scr = statistics.median(e[0].elapsed_time(e[1]) for e in pevs)
+        dec_t = statistics.median(e[1].elapsed_time(e[2]) for e in pevs)
         # counts for the byte model (untimed extra screen with count outputs)
         ucnt = torch.zeros((w.B, w.Hkv), dtype=torch.int32, device=dev)
         hcnt = torch.zeros((w.B, w.Hq), dtype=torch.int32, device=dev)
@@ -436,8 +515,8 @@ def run_eta(args):
         st = dec.device_status()
         if st != 0:
             raise RuntimeError(f"device status {st} after timed steps")
-        return {"ms": tot, "ms_screen": scr, "ms_decode": dec_t, "bytes": bm,
-                "clocks": clocks, "tau": (tau, stride, bias)}
+        return {"ms": tot, "ms_mean": sum(per_step) / len(per_step), "ms_screen": scr, "ms_decode": dec_t,
+                "bytes": bm, "clocks": clocks, "tau": (tau, stride, bias)}
 
     def time_dense():
         for _ in range(args.warmup):
@@ -451,7 +530,7 @@ def run_eta(args):
             dec.dense(dw.q, dw.K, dw.V, w.n)
             evs[i][1].record(stream)
         torch.cuda.synchronize()
-        return sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        return statistics.median(e[0].elapsed_time(e[1]) for e in evs)
 
     def time_e2e(tau, stride, bias):
         """Public API (EtaDecoder.step) with q from pinned host memory and the
@@ -479,7 +558,7 @@ def run_eta(args):
             one()
             evs[i][1].record(stream)
         torch.cuda.synchronize()
-        ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+        ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
         h2d = q_pin.numel() * q_pin.element_size()
         d2h = out_pin.numel() * out_pin.element_size()
         return ms, h2d, d2h
@@ -494,7 +573,9 @@ def run_eta(args):
     achieved = bm["decode_kernel"] / (ms_dec * 1e-3) / 1e9
     line = {
         "metric": "sparse decode queries/s", "value": value, "unit": "queries/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "ms_per_step_mean": max_over_ranks(main["ms_mean"], world), "step_time": "median of the timed steps",
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": {"bf16": "bf16", "fp8": "fp8", "f32": "f32"}[w.dtype],
         "data": "synthetic (seeded Philox4x32-10 + Box-Muller normals, shaped like the pages' decode workloads)",
         "config": {"workload": w.name, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "head_dim": w.d,
@@ -604,6 +685,8 @@ def cpu_baseline(w, args, dw):
 
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args))
     if args.impl == "reference":
         run_reference(args)
     else:

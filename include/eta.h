@@ -388,9 +388,10 @@ ETA_API eta_status_t eta_block_stats(const eta_shape_t* shape, const eta_params_
  * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and
  * without any device allocation. The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory when they
- * decode (a CUDA graph being captured, a serving engine whose memory plan is
- * frozen at start-up, a host framework that owns every allocation, a
- * real-time loop that must not enter an allocator).
+ * decode: a serving engine whose memory plan is frozen at start-up, a host
+ * framework that owns every allocation and hands out only finished tensors,
+ * a real-time loop that must not enter an allocator (cudaMalloc may
+ * synchronise the device and has no latency bound).
  *
  * The scratch is a fixed array of ETA_STATIC_SCRATCH_BYTES inside the library,
  * one per device that loads it, held until the process exits. Shapes whose

@@ -132,6 +132,14 @@ eta_status_t check_sub_blocks(const eta_shape_t* s, const eta_params_t* p, bool 
   return ETA_OK;
 }
 
+// Store rows (token rows of the K cache or pool) that a kernel addresses with
+// a 32-bit row index: the metadata builder's block rows, like the decode's.
+eta_status_t check_store_rows(const eta_shape_t* s, int64_t pool_pages) {
+  const int64_t rows = pool_pages > 0 ? pool_pages * s->n_kv_heads * s->block_size
+                                      : static_cast<int64_t>(s->batch) * s->n_kv_heads * s->capacity;
+  return rows > static_cast<int64_t>(INT32_MAX) ? ETA_ERR_UNSUPPORTED : ETA_OK;
+}
+
 // Shapes the decode kernel can stage (two stages of a K and a V block plus its
 // fixed shared memory) and index (prefix table and partial counters of B*Hkv
 // entries).
@@ -145,13 +153,8 @@ eta_status_t check_decode_shape(const eta_shape_t* s, bool dense, int64_t pool_p
                        static_cast<size_t>(BH + 1) * 4 + 64;
   const size_t need = 2 * (2 * tile + 32) + fixed;
   if (need + 1024 > static_cast<size_t>(device_max_smem_optin())) return ETA_ERR_UNSUPPORTED;
-  // bf16 K/V with bf16 q take the tensor-core kernel, whose TMA tensor copies
-  // address cache rows with 32-bit coordinates
-  const int64_t store_rows = pool_pages > 0 ? pool_pages * s->n_kv_heads * s->block_size
-                                           : static_cast<int64_t>(BH) * s->capacity;
   // the kernels address store rows with 32-bit integers (TMA coordinates too)
-  if (store_rows > static_cast<int64_t>(INT32_MAX)) return ETA_ERR_UNSUPPORTED;
-  return ETA_OK;
+  return check_store_rows(s, pool_pages);
 }
 
 // A paged pool: a block table and at least one page.
@@ -310,6 +313,7 @@ ETA_API eta_status_t eta_build_block_meta(const eta_shape_t* shape, const void* 
                                           int64_t blk_end, eta_meta_t meta, eta_stream_t stream) {
   ETA_TRY(check_shape(shape));
   ETA_TRY(check_meta(meta));
+  ETA_TRY(check_store_rows(shape, 0));
   if (k == nullptr || !aligned(k, 16)) return ETA_ERR_INVALID_ARG;
   const int64_t nb_cap = shape->capacity / shape->block_size;
   if (blk_begin < 0 || blk_end > nb_cap || blk_begin > blk_end) return ETA_ERR_INVALID_ARG;
@@ -518,6 +522,7 @@ ETA_API eta_status_t eta_build_block_meta_paged(const eta_shape_t* shape, const 
   ETA_TRY(check_shape(shape));
   ETA_TRY(check_meta(meta));
   ETA_TRY(check_pages(pages));
+  ETA_TRY(check_store_rows(shape, pages.num_pages));
   if (k_pool == nullptr || !aligned(k_pool, 16)) return ETA_ERR_INVALID_ARG;
   const int64_t nb_cap = shape->capacity / shape->block_size;
   if (blk_begin < 0 || blk_end > nb_cap || blk_begin > blk_end) return ETA_ERR_INVALID_ARG;

@@ -2,14 +2,13 @@
 // fixed device array inside this library, for callers that cannot allocate
 // device memory at call time.
 //
-// Who needs it: a caller recording the decode into a CUDA graph or running
-// under a frozen memory plan (serving engines that reserve all device memory
-// at start-up and forbid later cudaMalloc), code embedded in a host framework
-// that owns every allocation and hands out only tensors, and real-time loops
-// that must not call into an allocator (cudaMalloc can synchronise the device
-// and its latency is unbounded). Such callers still own their inputs and
-// outputs; only the per-call scratch (admitted-block lists, split partials,
-// status word) moves into the library.
+// Who needs it: a caller running under a frozen memory plan (serving engines
+// that reserve all device memory at start-up and forbid later cudaMalloc),
+// code embedded in a host framework that owns every allocation and hands out
+// only tensors, and real-time loops that must not call into an allocator
+// (cudaMalloc can synchronise the device and its latency is unbounded). Such
+// callers still own their inputs and outputs; only the per-call scratch
+// (admitted-block lists, split partials, status word) moves into the library.
 //
 // The scratch is one file-scope __device__ array of kStaticScratchBytes. Every
 // GPU that loads the library holds it until the process exits. All calls on a

@@ -117,6 +117,12 @@ def test_argument_validation_before_launch():
     assert L.eta_build_block_meta(ctypes.byref(s), a16, -1, 3, meta, None) == 1
     assert L.eta_build_block_meta(ctypes.byref(s), a16, 0, 33, meta, None) == 1
     assert L.eta_build_block_meta(ctypes.byref(s), a16, 5, 5, meta, None) == 0      # empty range: no-op
+    # more cache (or pool) rows than a 32-bit row index reaches: unsupported, for the builders too
+    big = _shape(batch=128, n_q_heads=16, n_kv_heads=16, block_size=16, capacity=1 << 20)
+    assert L.eta_build_block_meta(ctypes.byref(big), a16, 0, 1, meta, None) == 2
+    assert L.eta_build_block_meta_paged(ctypes.byref(s), a16, binding.Pages(1 << 20, 1 << 26), 0, 1, meta,
+                                        None) == 2
+    assert L.eta_build_block_meta_paged(ctypes.byref(s), a16, binding.Pages(1 << 20, 64), 0, 0, meta, None) == 0
     assert L.eta_predict_tau(ctypes.byref(s), None, a16, a16, a16, None) == 1
     st = ctypes.c_int(0)
     assert L.eta_read_device_status(None, None, ctypes.byref(st)) == 1

@@ -2,7 +2,11 @@
 bytes of the admitted union blocks with the partial last block counted by its
 valid rows, metadata of the screened blocks (r columns per block with the
 sub-block envelope), and the split partials only for segments that cross
-thread-block ranges."""
+thread-block ranges. The dense K+V bytes are pinned to the cache sizes printed
+in the pages' Table 5 (thelatestinai.com)."""
+import json
+import os
+
 import numpy as np
 import pytest
 
@@ -54,3 +58,18 @@ def test_partials_only_for_segments_crossing_ranges():
     m2 = bench.byte_model(w, small, hcnt, S=148)
     b2 = bench.byte_model(w, small, hcnt, S=1)
     assert m2["decode_kernel"] - b2["decode_kernel"] == 2 * partial   # segment 1 has 2 entries -> 2 parts
+
+
+def test_dense_kv_bytes_match_table5_cache_sizes():
+    """Table 5's KV column (H_Q 32, H_KV 4, d_h 64, fp16): 2 GB at B 32 and 64K
+    tokens, doubling with L and with B. The byte model's dense K+V bytes of the
+    same shapes in a 2-byte dtype must be exactly those sizes (GiB)."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "table5_kv_bytes.json")
+    g = json.load(open(path))
+    for row in g["rows"]:
+        w = _w(B=row["B"], Hq=32, Hkv=g["h_kv"], d=g["head_dim"], n=row["L"], bs=64)
+        ucnt = np.full((w.B, w.Hkv), w.nb, np.int64)
+        hcnt = np.full((w.B, w.Hq), w.nb, np.int64)
+        m = bench.byte_model(w, ucnt, hcnt, S=148)
+        assert m["dense_kv"] == row["gib"] << 30, row
+        assert m["kv"] == m["dense_kv"]           # every block admitted: the dense bytes

@@ -42,12 +42,39 @@ def test_two_rank_max_and_throughput():
     assert res[0][2] == pytest.approx(2 * 256 / 2e-3)
 
 
-def test_reference_arm_on_non_zero_rank_does_nothing(monkeypatch, capsys):
+def test_bench_gpus_two_starts_two_ranks():
+    """`bench.py --gpus 2` run as a plain process starts two ranks itself (the
+    reference arm runs on CPU: rank 0 prints the only line, with n_gpus 2)."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--config", "1", "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
+                       timeout=300, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+
+
+def test_rank_count_must_equal_gpus(monkeypatch):
     import bench
-    monkeypatch.setenv("RANK", "1")
-    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("WORLD_SIZE", "1")
 
     class A:
-        config, batch, density, steps, warmup = 3, None, 0.38, 1, 1
-    bench.run_reference(A())
-    assert capsys.readouterr().out == ""
+        gpus = 2
+    with pytest.raises(SystemExit):
+        bench.dist_setup(A())
+    with pytest.raises(SystemExit):
+        bench.run_reference(A())
+
+
+def test_relaunch_command_keeps_the_arguments():
+    import bench
+    cmd = bench.relaunch_command(["--gpus", "4", "--steps", "3"], 4, 29500)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "3"]

@@ -1,11 +1,13 @@
 """The allocation-free decode entry point (eta_decode_sparse_static).
 
-Callers that cannot allocate device memory while decoding (graph capture,
-frozen serving memory plans, host frameworks that own all allocations,
-real-time loops) call this variant, which keeps its scratch in a fixed device
-array inside the library. It must give the same result as eta_decode_sparse
-with a caller workspace, call after call (the shared scratch keeps the
-previous call's contents), and reject shapes larger than its scratch.
+Some callers cannot allocate device memory while they decode: a serving engine
+whose memory plan is fixed at start-up, a host framework that owns every
+allocation, a real-time loop that must not enter an allocator. They call this
+variant, which keeps its scratch in a fixed device array inside the library.
+It runs the same kernels as eta_decode_sparse with a caller workspace, so on
+the same inputs its outputs, counts and lists must be identical bit for bit,
+call after call (the shared scratch keeps the previous call's contents), and
+it must reject shapes larger than its scratch.
 
 This file is collected last on purpose, so a run that stops at the first
 failure has already run every other test."""
@@ -19,8 +21,6 @@ from learned_block_sparse_b200.workload import DeviceWorkload
 
 pytestmark = pytest.mark.gpu
 
-TOL_BF16 = 2e-3
-
 
 def _thresholds(dw, density):
     tau, stride, bias = dw.calibrate(density)
@@ -31,6 +31,14 @@ def _thresholds(dw, density):
     return tau, stride
 
 
+def _lists(w, dev):
+    nb_cap = w.capacity // w.bs
+    return dict(active_idx=torch.full((w.B, w.Hq, nb_cap), -1, dtype=torch.int32, device=dev),
+                active_cnt=torch.full((w.B, w.Hq), -1, dtype=torch.int32, device=dev),
+                union_list=torch.zeros((w.B, w.Hkv, nb_cap), dtype=torch.int32, device=dev),
+                union_cnt=torch.full((w.B, w.Hkv), -1, dtype=torch.int32, device=dev))
+
+
 def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
     w = synth.WORKLOADS[3].replace(B=2, Hq=8, Hkv=2, n=32 * 150 + 5)
     dw = DeviceWorkload(w)
@@ -39,17 +47,22 @@ def test_static_scratch_matches_workspace_entry_point_on_consecutive_calls():
     for density in (0.38, 0.2):              # two calls in a row, different admitted sets
         tau, stride = _thresholds(dw, density)
         ref = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dw.device)
-        binding.decode_sparse(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, w.n, tau, stride, ref, dec.ws)
+        ref_lists = _lists(w, dw.device)
+        binding.decode_sparse(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, w.n, tau, stride, ref, dec.ws,
+                              **ref_lists)
         out = torch.full_like(ref, float("nan"))
+        got_lists = _lists(w, dw.device)
         status = torch.full((1,), -1, dtype=torch.int32, device=dw.device)
-        cnt = torch.full((w.B, w.Hq), -1, dtype=torch.int32, device=dw.device)
         binding.decode_sparse_static(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, w.n, tau, stride, out,
-                                     device_status=status, active_cnt=cnt)
+                                     device_status=status, **got_lists)
         torch.cuda.synchronize()
+        assert dec.device_status() == 0
         assert int(status.item()) == 0
-        assert torch.isfinite(out).all()
-        assert float((out - ref).abs().max()) <= TOL_BF16
-        assert int(cnt.min()) >= 1
+        # same kernels, same inputs: the same bits
+        assert torch.equal(out, ref)
+        for key in ref_lists:
+            assert torch.equal(got_lists[key], ref_lists[key]), key
+        assert int(got_lists["active_cnt"].min()) >= 1
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
