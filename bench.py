@@ -162,107 +162,90 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+_SAMPLER = r"""
+import sys, time
+import pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByUUID(sys.argv[1])
+mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+rd = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+    pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+period = float(sys.argv[2])
+with open(sys.argv[3], "w", buffering=1) as f:
+    while True:
+        f.write("%.6f %d %d %d\n" % (time.monotonic(), pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                       mx, rd(h)))
+        time.sleep(period)
+"""
+
+
 class ClockSampler:
     """SM clock and clock-event reasons sampled DURING the timed region.
 
-    A thread polls NVML about once a millisecond from start() to stop(), so
-    that a timed region of a few tens of milliseconds still gets tens of
-    samples; when NVML is not importable it falls back to nvidia-smi's
-    20 ms loop. The device is found by its UUID (CUDA and NVML may number
-    GPUs differently)."""
+    A separate process polls NVML about once a millisecond (an NVML query
+    takes ~1 us) and stamps each sample with the system-wide monotonic clock;
+    start() returns once it is sampling, stop() keeps the samples taken between
+    the two calls. A separate process, so the benchmark's own thread never
+    delays the sampling. The device is found by its UUID (CUDA and NVML may
+    number GPUs differently)."""
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
-    SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-                  "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int, period_s: float = 0.001):
         self.dev = device_index
         self.period = period_s
-        self.samples = []          # (sm_mhz, max_mhz, reasons bitmask)
-        self.thread = None
         self.proc = None
         self.path = None
-        self.source = None
-        self._stop = False
-
-    def _nvml_handle(self):
-        import pynvml
-        pynvml.nvmlInit()
-        props = torch.cuda.get_device_properties(self.dev)
-        try:
-            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
-        except Exception:
-            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
-            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
-            nv, h = self._nvml_handle()
-            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            read = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                nv.nvmlDeviceGetCurrentClocksThrottleReasons
-
-            def loop():
-                while not self._stop:
-                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx, int(read(h))))
-                    time.sleep(self.period)
-            import threading
-            self.thread = threading.Thread(target=loop, daemon=True)
-            self.source = "nvml, ~1 ms polling"
-            self.thread.start()
-            return
-        except Exception:
-            self.thread = None
-        try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+            fd, self.path = tempfile.mkstemp(suffix=".txt")
             os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.SMI_FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            self.source = "nvidia-smi -lms 20"
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, uuid, str(self.period), self.path],
+                                         stderr=subprocess.DEVNULL)
+            deadline = time.monotonic() + 20.0
+            while time.monotonic() < deadline and self.proc.poll() is None:
+                if os.path.getsize(self.path) > 0:
+                    break
+                time.sleep(0.01)
+            if self.proc.poll() is not None or os.path.getsize(self.path) == 0:
+                self.stop()
+                self.proc = None
+                return
         except Exception:
             self.proc = None
-
-    def _smi_samples(self):
-        names = [nm for nm, _ in self.REASONS[:4]]
-        bits = dict(self.REASONS)
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm, mx = float(parts[1]), float(parts[2])
-                except ValueError:
-                    continue
-                mask = 0
-                for nm, val in zip(names, parts[5:9]):
-                    if val.lower() == "active":
-                        mask |= bits[nm]
-                self.samples.append((sm, mx, mask))
-        os.unlink(self.path)
+            return
+        self.t0 = time.monotonic()
 
     def stop(self):
-        if self.thread is not None:
-            self._stop = True
-            self.thread.join(timeout=5)
-        elif self.proc is not None:
-            time.sleep(0.05)
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self._smi_samples()
-        else:
+        if self.proc is None:
             return None
-        if not self.samples:
+        self.t1 = time.monotonic()
+        time.sleep(2 * self.period)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        samples = []
+        with open(self.path) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) != 4:
+                    continue
+                t, sm, mx, mask = float(parts[0]), int(parts[1]), int(parts[2]), int(parts[3])
+                if self.t0 is not None and self.t0 <= t <= self.t1:
+                    samples.append((sm, mx, mask))
+        os.unlink(self.path)
+        if not samples:
             return None
-        reasons = sorted({nm for (_, _, m) in self.samples for nm, bit in self.REASONS if m & bit})
-        sm = [x[0] for x in self.samples]
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
-                "sm_mhz_min": min(sm), "reasons": reasons, "samples": len(sm), "source": self.source}
+        reasons = sorted({nm for (_, _, m) in samples for nm, bit in self.REASONS if m & bit})
+        sm = [x[0] for x in samples]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in samples), "sm_mhz_min": min(sm),
+                "reasons": reasons, "samples": len(sm),
+                "source": "NVML polled ~1 kHz by a separate process, samples inside the timed region"}
 
 
 # ------------------------------------------------------------ byte models

@@ -412,6 +412,22 @@ ETA_API eta_status_t eta_decode_sparse_static(const eta_shape_t* shape, const et
                                               const eta_screen_out_t* extra, int32_t* device_status,
                                               eta_stream_t stream);
 
+/*
+ * eta_test_withhold_copy — test hook of the device-timeout path; the paper has
+ * no counterpart. The next decode launch in this process (any eta_decode_*
+ * call) leaves the K/V copy of one admitted block unissued: position
+ * `position` (0-based) of the first thread block's range. The consumer warp
+ * that owns that block waits for it up to the library's device wait limit
+ * (2 s), then every warp of that thread block stops, the copies already
+ * issued are allowed to land, and the call records ETA_ERR_DEVICE_TIMEOUT in
+ * the workspace status word; its outputs are then undefined. Nothing faults
+ * and the context stays usable: read (and so clear) the status with
+ * eta_read_device_status, and the next call computes normally. A position
+ * past the end of that range withholds nothing; a negative position disarms
+ * the hook. Always returns ETA_OK. Not for production use.
+ */
+ETA_API eta_status_t eta_test_withhold_copy(int64_t position);
+
 /* Synchronise `stream`, read the workspace's device status word into *status
  * (host pointer) and clear it (the whole header when it was not ETA_OK).
  * Returns ETA_ERR_CUDA if the copy fails. */

@@ -105,6 +105,8 @@ def _load():
     L.eta_decode_dense_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_block_stats.restype = st
     L.eta_block_stats.argtypes = [P(Shape), P(Params), vp, vp, i64, vp, i64, vp, vp, vp, vp]
+    L.eta_test_withhold_copy.restype = st
+    L.eta_test_withhold_copy.argtypes = [i64]
     L.eta_decode_screened.restype = st
     L.eta_decode_screened.argtypes = [P(Shape), P(Params), vp, vp, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_decode_dense.restype = st
@@ -123,7 +125,8 @@ EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta
             "eta_decode_screened", "eta_decode_dense", "eta_read_device_status", "eta_decode_sparse_static",
             "eta_screen_predict", "eta_decode_sparse_predict", "eta_screen_ragged", "eta_decode_sparse_ragged",
             "eta_decode_screened_ragged", "eta_decode_dense_ragged", "eta_build_block_meta_paged",
-            "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged", "eta_block_stats")
+            "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged", "eta_block_stats",
+            "eta_test_withhold_copy")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -357,6 +360,13 @@ def decode_sparse_static(shape: Shape, params: Params, q, k, v, meta, n_tokens: 
                                         Meta(*(m.data_ptr() for m in meta)), n_tokens, _ptr(tau), tau_batch_stride,
                                         _ptr(out), ctypes.byref(so) if so is not None else None,
                                         _ptr(device_status), _stream(stream)), "eta_decode_sparse_static")
+
+
+def withhold_next_copy(position: int) -> None:
+    """Test hook: the next decode launch leaves the copy of one admitted block
+    (position `position` of the first thread block's range) unissued, so its
+    bounded wait runs out and the call reports ETA_ERR_DEVICE_TIMEOUT."""
+    _check(lib.eta_test_withhold_copy(position), "eta_test_withhold_copy")
 
 
 def read_device_status(ws: torch.Tensor, stream=None) -> int:

@@ -236,6 +236,10 @@ eta_status_t check_common_decode(const eta_shape_t* s, const eta_params_t* p, co
   return ETA_OK;
 }
 
+// Test hook of the device-timeout path (eta_test_withhold_copy): the position
+// the next decode launch leaves unarmed, -1 for none.
+std::atomic<int64_t> g_withhold{-1};
+
 eta_status_t do_decode(const eta_shape_t* s, const eta_params_t* p, const void* q, const void* k, const void* v,
                        int64_t n, const float* tau, int64_t tau_stride, float* out, const Workspace& w,
                        cudaStream_t st, bool dense, const int32_t* seq_lens = nullptr,
@@ -257,6 +261,7 @@ eta_status_t do_decode(const eta_shape_t* s, const eta_params_t* p, const void* 
   c.ws = w;
   c.S = resolve_splits(p);
   c.dense = dense;
+  c.withhold = g_withhold.exchange(-1);
   return from_cuda(launch_decode(c, st));
 }
 
@@ -586,6 +591,11 @@ ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_
   ETA_TRY(check_workspace(shape, params, workspace, ws_bytes, &L));
   return do_decode(shape, params, q, k_pool, v_pool, max_tokens, tau, tau_batch_stride, out, ws_carve(workspace, L),
                    stream, true, seq_lens, &pages);
+}
+
+ETA_API eta_status_t eta_test_withhold_copy(int64_t position) {
+  g_withhold.store(position < 0 ? -1 : position);
+  return ETA_OK;
 }
 
 ETA_API eta_status_t eta_block_stats(const eta_shape_t* shape, const eta_params_t* params, const void* q,

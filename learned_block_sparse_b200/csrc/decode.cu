@@ -137,7 +137,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
   int it = 0;
   for (int64_t p = lo; p < hi; ++p, ++it) {
     const int st = it % NST;
-    const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, a.status);
+    // the warp's lanes reduce together: all of them process the stage or none
+    const bool ok =
+        __all_sync(kFull, mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, a.status));
     if (ok) {
       const int4 inf = s_info[st];
       const unsigned char* kt = s_tiles + static_cast<size_t>(st) * 2 * tile_bytes;
@@ -229,7 +231,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const DecodeArgs
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&s_empty[st]);
+    if (ok && lane == 0) mbar_arrive(&s_empty[st]);  // a stage whose wait failed is not released
 
     if (p + 1 == seg_end || p + 1 == hi) {
       // ---- emit this range's partial for segment `cur`

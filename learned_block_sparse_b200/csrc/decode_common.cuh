@@ -30,6 +30,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
   int gate;  // ETA_GATE_SIGMOID or ETA_GATE_HARD
   float beta, qscale;
+  int64_t withhold;  // test hook: position of thread block 0's range whose copy is never armed (-1: none)
 };
 
 __device__ __forceinline__ int find_seg(const int32_t* pre, int BH, int64_t p) {
@@ -180,6 +181,15 @@ __device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int
 // entries at a time, one batch ahead. A stage's r-th reuse waits for the
 // consumer release that completed the empty barrier's phase r-1; the round a
 // stage serves is then published in s_round (when given) before it is armed.
+//
+// Abort protocol. Consumers release a stage only after its full barrier
+// completed, so a stage is never re-armed while its copies are in flight.
+// Once any warp of the thread block has given up (s_abort), the producer arms
+// nothing more; whatever happened, before returning it waits (bounded) until
+// the copies of the last armed use of every stage have landed, so the thread
+// block never exits with a copy in flight. a.withhold (a test hook) leaves one
+// position of thread block 0 unarmed, so that its consumer's bounded wait runs
+// out and the call ends with ETA_ERR_DEVICE_TIMEOUT.
 template <int G, bool DENSE, int kMaxPL, typename SegOf, typename Pre, typename Issue>
 __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, int64_t hi, int NST,
                                               uint64_t* s_empty, int4* s_info, int* s_abort, SegOf seg_of,
@@ -221,7 +231,9 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
   uint32_t e_cur, e_nxt = 0;
   fetch(lo + lane, seg_cur, e_cur);
   int issued = 0;    // this lane: 1 + the last position (relative to lo) it armed
+  int held = -1;     // the position left unarmed by the test hook
   int aborted = 0;
+  volatile int* abort_flag = s_abort;
   for (int64_t base = lo; base < hi && !aborted; base += 32) {
     finish(base + lane, seg_cur, e_cur, rows_cur, row_cur);
     if (base + 32 < hi) fetch(base + 32 + lane, seg_nxt, e_nxt);
@@ -237,6 +249,7 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
         const int st = it % NST;
         const int round = it / NST;
         if (round > 0 && !mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, a.status)) aborted = 1;
+        if (!aborted && *abort_flag) aborted = 1;  // a consumer gave up: arm nothing more
         if (!aborted) {
           const int blk = static_cast<int>(e_i >> 8);
           int rows = rows_i;
@@ -246,7 +259,8 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
           }
           if (s_round != nullptr) s_round[st] = round;  // this stage now serves round `round`
           s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
-          if (rows == 0) mbar_arrive(&s_full[st]);
+          if (blockIdx.x == 0 && it == a.withhold) held = it;   // test hook: never armed
+          else if (rows == 0) mbar_arrive(&s_full[st]);
           else issue(st, row_i, rows);
           issued = it + 1;
         }
@@ -256,9 +270,14 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
     seg_cur = seg_nxt;
     e_cur = e_nxt;
   }
-  if (aborted && lane < PL) {
-    // let the copies this lane armed land before the thread block can exit
-    for (int j = issued - 1; j >= 0 && j >= issued - NST; j -= PL) {
+  // Positions >= last - NST are the last armed use of their stage (last = 1 +
+  // the last position any lane armed): wait until each of this lane's has
+  // completed, so no copy is in flight when the thread block exits. Earlier
+  // positions completed before their stage was re-armed.
+  const int last = __reduce_max_sync(kFull, issued);
+  if (lane < PL) {
+    for (int j = issued - 1; j >= 0 && j >= last - NST; j -= PL) {
+      if (j == held) continue;
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
       }
@@ -301,6 +320,7 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.q_dtype = s.q_dtype;
   a.beta = c.beta;
   a.gate = c.gate;
+  a.withhold = c.withhold;
   a.qscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.head_dim)));
   return a;
 }

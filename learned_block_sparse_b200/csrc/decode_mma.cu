@@ -589,9 +589,15 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     // it itself, and the extra wait is skipped.)
     bool ok = round == 0 || (NST % kMW) == 0 || wait_value_bounded(s_round + st, round, s_abort, a.status);
     ok = ok && mbar_wait_bounded(&s_full[st], static_cast<uint32_t>(round & 1), s_abort, a.status);
-    if (ok) process(st, s_info[st]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&s_empty[st]);
+    // the tile math is warp-synchronous: the whole warp processes the stage or
+    // none of it; a stage whose wait failed is not released (its copies may
+    // still be in flight), and the producer stops once it sees the abort
+    ok = __all_sync(kFull, ok);
+    if (ok) {
+      process(st, s_info[st]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[st]);
+    }
   }
 }
 

@@ -113,6 +113,7 @@ struct DecodeCall {
   Workspace ws;
   int S;                   // number of work ranges (grid size)
   bool dense;
+  int64_t withhold = -1;   // test hook (eta_test_withhold_copy): unarmed position of thread block 0
 };
 cudaError_t launch_decode(const DecodeCall& c, cudaStream_t st);
 

@@ -117,8 +117,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   };
   // the first ring of tiles does not depend on the queries: start it now
   const int first = my_tiles < NST ? my_tiles : NST;
-  if (warp == CW && lane == 0)
+  int issued = 0;  // producer lane: 1 + the last tile it armed
+  if (warp == CW && lane == 0) {
     for (int it = 0; it < first; ++it) issue_tile(it);
+    issued = first;
+  }
   screen_prologue<D, G, 32, false>(a, sm, b, kvh, NT);  // ends with __syncthreads
   const bool tau_later = a.W != nullptr;
 
@@ -134,23 +137,13 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   } else if (warp == CW) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = first;
-      bool aborted = false;
-      for (int it = first; it < my_tiles && !aborted; ++it) {
+      volatile int* abort_flag = s_abort;
+      for (int it = first; it < my_tiles; ++it) {
         const int st = it % NST, round = it / NST;
-        if (!mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status)) {
-          aborted = true;
-          break;
-        }
+        // a consumer that gave up does not release its stage: stop arming
+        if (!mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status) || *abort_flag) break;
         issue_tile(it);
         issued = it + 1;
-      }
-      if (aborted) {  // let the copies already issued land before exiting
-        for (int j = max(0, issued - NST); j < issued; ++j) {
-          const uint64_t tstart = global_timer_ns();
-          while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - tstart < kWaitLimitNs) {
-          }
-        }
       }
     }
   } else {
@@ -162,7 +155,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
       const int unit = (t0 + it) * 32 + lane;
       const bool valid = unit < units;
       const float M = __ldg(mx + (valid ? unit : units - 1));  // units >= 1 here (this CTA has a tile)
-      const bool ok = mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status);
+      const bool ok =
+          __all_sync(kFull, mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status));
       float dg[G], vg[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) dg[g] = vg[g] = 0.0f;
@@ -216,7 +210,7 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[st]);
+      if (ok && lane == 0) mbar_arrive(&s_empty[st]);  // a stage whose wait failed is not released
       if (!tau_waited) {
         tau_ok = mbar_wait_bounded(s_tau, 0u, s_abort, status);
         tau_waited = true;
@@ -225,6 +219,15 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
     }
   }
   __syncthreads();
+  if (warp == CW && lane == 0 && *reinterpret_cast<volatile int*>(s_abort)) {
+    // a wait gave up: let the copies of the last use of every stage land before
+    // the thread block can exit (earlier uses completed before their re-arm)
+    for (int j = max(0, issued - NST); j < issued; ++j) {
+      const uint64_t tstart = global_timer_ns();
+      while (!mbar_try_wait(&s_full[j % NST], (j / NST) & 1) && global_timer_ns() - tstart < kWaitLimitNs) {
+      }
+    }
+  }
   screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, rb, NT);
 }
 

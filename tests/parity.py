@@ -166,3 +166,67 @@ def compare(w, gpu, orc, heads, check_lists=True):
             g_u = gpu["union_list"][b, kvh, :ucnt].astype(np.int64) & 0xffffffff
             assert np.array_equal(g_u, packed), f"union list mismatch at ({b},{kvh})"
     return max_err
+
+
+def host_rows(w, q_host, batches, needles=None):
+    """Host K and V of the given batch rows only, {(b, kv head): [capacity][d]}:
+    the oracle's inputs for full-size workloads whose whole cache stays on the
+    device (the same seeded bytes the device copy was filled with)."""
+    K, V = {}, {}
+    for b in sorted(set(batches)):
+        for which, dst in (("k", K), ("v", V)):
+            buf = torch.empty((1, w.Hkv, w.capacity, w.d), dtype=w.torch_dtype)
+            synth.fill_kv(w, q_host, which, buf, b, b + 1, needles)
+            for h in range(w.Hkv):
+                dst[(b, h)] = buf[0, h]
+    return K, V
+
+
+def oracle_rows(w, q_host, K_host, V_host, meta, lens, tau_bh, dense=False, heads=None):
+    """Per-row-length oracle: row b screens, gates and attends as a call with
+    n = lens[b] (its own current token and forced trailing blocks)."""
+    qf = oracle.to_f32(q_host)
+
+    def one(b, hq):
+        n_b = lens[b]
+        nb_b = (n_b + w.bs - 1) // w.bs
+        kvh = hq // w.G
+        if dense:
+            lst, sc = np.arange(nb_b, dtype=np.int32), None
+            t = float("-inf")
+        else:
+            mu, var, mx = meta[(b, kvh)]
+            t = tau_bh(b, hq)
+            lst, sc = oracle.screen_head(qf[b, hq], mu, var, mx, nb_b, w.n_local, w.z, t)
+        o = oracle.attend_head(K_host[b, kvh], V_host[b, kvh], w.bs, n_b, qf[b, hq], lst, t, w.beta)
+        return (b, hq), (lst, sc, o)
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.Hq)]
+    return dict(pmap(one, heads))
+
+
+def compare_rows(w, lens, outs, out, orc, check_lists=True):
+    """Assert per-row parity: outputs within tolerance; counts, lists, scores and
+    GQA unions bit-exact; no score written past a row's screened blocks."""
+    tol = TOL[w.dtype]
+    got = {k: v.cpu().numpy() for k, v in outs.items()} if check_lists else {}
+    o_gpu = out.cpu().numpy()
+    for (b, hq), (lst, sc, o) in orc.items():
+        err = float(np.max(np.abs(o_gpu[b, hq].astype(np.float64) - o)))
+        assert err <= tol, f"output of row {b} (n={lens[b]}) head {hq}: {err:.3g}"
+        if not check_lists:
+            continue
+        cnt = int(got["active_cnt"][b, hq])
+        assert cnt == len(lst) and np.array_equal(got["active_idx"][b, hq, :cnt], lst), (b, hq, lens[b])
+        if "scores" in got:
+            ns_b = max(0, (lens[b] + w.bs - 1) // w.bs - w.n_local)
+            assert np.array_equal(got["scores"][b, hq, :ns_b].view(np.int32), sc.view(np.int32)), (b, hq)
+            assert np.all(np.isnan(got["scores"][b, hq, ns_b:w.n_screened])), "scores past the row were written"
+    if not check_lists:
+        return
+    for (b, kvh) in sorted({(b, hq // w.G) for (b, hq) in orc}):
+        nb_b = (lens[b] + w.bs - 1) // w.bs
+        idx, mask = oracle.union_lists([orc[(b, kvh * w.G + g)][0] for g in range(w.G)], nb_b)
+        ucnt = int(got["union_cnt"][b, kvh])
+        packed = (idx.astype(np.int64) << 8) | mask.astype(np.int64)
+        assert ucnt == len(idx)
+        assert np.array_equal(got["union_list"][b, kvh, :ucnt].astype(np.int64) & 0xffffffff, packed)

@@ -1,15 +1,17 @@
 """Paged KV pools (eta_*_paged): the K and V blocks of a contiguous cache are
-scattered into randomly permuted pages of a pool; metadata built from the pool
-and every decode result (lists, thresholds, outputs, dense outputs) must equal
-the contiguous per-row-length calls bit for bit (those are checked against the
-oracle in test_gpu_ragged.py). A page index outside the pool is reported in the
-device status word and never read."""
+scattered into randomly permuted pages of a pool. Metadata built from the pool
+and every decode result (thresholds, lists, scores, unions, outputs, dense
+outputs) are checked against the oracle run row by row on the same seeded
+cache (bit-exact decisions, outputs within 2e-3 / 1e-5), and must also equal
+the contiguous per-row-length calls bit for bit. A page index outside the pool
+is reported in the device status word and never read."""
 import numpy as np
 import pytest
 import torch
 
 from learned_block_sparse_b200 import binding, synth
 from learned_block_sparse_b200.workload import DeviceWorkload
+from tests import parity
 
 pytestmark = pytest.mark.gpu
 
@@ -49,7 +51,8 @@ def _outs(w):
     return dict(active_idx=torch.full((w.B, w.Hq, nb_cap), -1, dtype=torch.int32, device="cuda"),
                 active_cnt=torch.zeros((w.B, w.Hq), dtype=torch.int32, device="cuda"),
                 union_list=torch.zeros((w.B, w.Hkv, nb_cap), dtype=torch.int32, device="cuda"),
-                union_cnt=torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda"))
+                union_cnt=torch.zeros((w.B, w.Hkv), dtype=torch.int32, device="cuda"),
+                scores=torch.full((w.B, w.Hq, nb_cap), float("nan"), dtype=torch.float32, device="cuda"))
 
 
 @pytest.mark.parametrize("dtype,Hq,Hkv,d,bs,mode", [
@@ -59,29 +62,46 @@ def _outs(w):
     ("f32", 4, 2, 64, 16, "predictor"),
     ("fp8", 8, 2, 128, 64, "const"),
 ])
-def test_paged_pool_equals_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
+def test_paged_pool_against_oracle_and_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
     w = synth.Workload("paged", dtype, 6, Hq, Hkv, d, bs * 50 + 3, bs, z=1.0, tau_mode=mode,
                        densities=(0.3,), seed=700 + bs + Hq, offset_std=synth.SQRT_HALF)
-    dw = DeviceWorkload(w)
+    dw = DeviceWorkload(w, keep_host=True)
     dec = dw.dec
     k_pool, v_pool, table, pages = _pool(dw, seed=bs)
-    # metadata from the pool = metadata from the contiguous cache
+    # metadata from the pool: the oracle's bit for bit (and the contiguous builder's)
     mu = torch.full_like(dec.mu, float("nan"))
     var = torch.full_like(dec.var, float("nan"))
     mx = torch.full_like(dec.maxnorm, float("nan"))
     nfull = w.n // w.bs
     binding.build_block_meta_paged(dec.shape, k_pool, table, pages, 0, nfull, mu, var, mx)
     torch.cuda.synchronize()
-    for a, b in ((mu, dec.mu), (var, dec.var)):
-        assert torch.equal(a[..., :nfull], b[..., :nfull])
-    assert torch.equal(mx[..., :nfull], dec.maxnorm[..., :nfull])
+    meta = parity.oracle_meta(w, dw.K_host)
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            o_mu, o_var, o_mx = meta[(b, h)]
+            assert np.array_equal(mu[b, h, :, :nfull].T.contiguous().cpu().numpy().view(np.int32),
+                                  o_mu.view(np.int32)), (b, h)
+            assert np.array_equal(var[b, h, :, :nfull].T.contiguous().cpu().numpy().view(np.int32),
+                                  o_var.view(np.int32)), (b, h)
+            assert np.array_equal(mx[b, h, :nfull].cpu().numpy().view(np.int32), o_mx.view(np.int32)), (b, h)
+    for a_, b_ in ((mu, dec.mu), (var, dec.var), (mx, dec.maxnorm)):
+        assert torch.equal(a_[..., :nfull], b_[..., :nfull])
 
-    seq = _lens(w, seed=bs + 1)
+    # thresholds from the oracle side
+    tau, stride, bias = parity.oracle_thresholds(w, dw.q_host, meta, 0.3, W=dw.W)
+    tau_arr = np.asarray(tau, np.float32)
     if mode == "predictor":
-        calib = dw.calibrate(0.3)
-        thr = dict(W=dw.W, bias=calib[2])
+        thr = dict(W=dw.W, bias=torch.as_tensor(bias, device="cuda"))
+
+        def tau_bh(b, h):
+            return float(tau_arr.reshape(w.B, w.Hq)[b, h])
     else:
-        thr = dict(tau=dw.calibrate(0.3)[0], tau_batch_stride=0)
+        thr = dict(tau=torch.as_tensor(tau_arr, device="cuda"), tau_batch_stride=0)
+
+        def tau_bh(b, h):
+            return float(tau_arr[h])
+    seq = _lens(w, seed=bs + 1)
+    lens = [int(x) for x in seq.cpu()]
     out_c = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
     out_p = torch.empty_like(out_c)
     tau_c = torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda")
@@ -89,25 +109,35 @@ def test_paged_pool_equals_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
     oc, op = _outs(w), _outs(w)
     extra_c = dict(tau_out=tau_c) if mode == "predictor" else {}
     extra_p = dict(tau_out=tau_p) if mode == "predictor" else {}
-    binding.decode_sparse_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, seq, w.n, out_c, dec.ws,
-                                 **thr, **extra_c, **oc)
     binding.decode_sparse_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, table, pages, (mu, var, mx), seq, w.n,
                                 out_p, dec.ws, **thr, **extra_p, **op)
     torch.cuda.synchronize()
     assert dec.device_status() == 0
-    for key in oc:
-        assert torch.equal(oc[key], op[key]), key
+    if mode == "predictor":
+        assert np.array_equal(tau_p.cpu().numpy().view(np.int32), tau_arr.reshape(w.B, w.Hq).view(np.int32))
+    orc = parity.oracle_rows(w, dw.q_host, dw.K_host, dw.V_host, meta, lens, tau_bh)
+    parity.compare_rows(w, lens, op, out_p, orc)
+    # the same call on the contiguous cache: the same bits
+    binding.decode_sparse_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, dec.meta, seq, w.n, out_c, dec.ws,
+                                 **thr, **extra_c, **oc)
+    torch.cuda.synchronize()
+    assert dec.device_status() == 0
+    for key in oc:   # bit patterns: unscreened score entries hold NaN on both sides
+        assert torch.equal(oc[key].view(torch.int32), op[key].view(torch.int32)), key
     if mode == "predictor":
         assert torch.equal(tau_c, tau_p)
     assert torch.equal(out_c, out_p)
-    # the dense pass over the pool
+
+    # the dense pass over the pool: plain softmax attention per row, as the oracle's
     dense_c = torch.empty_like(out_c)
     dense_p = torch.empty_like(out_c)
-    binding.decode_dense_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, seq, w.n, None, 0, dense_c, dec.ws)
     binding.decode_dense_paged(dec.shape, dec.params, dw.q, k_pool, v_pool, table, pages, seq, w.n, None, 0,
                                dense_p, dec.ws)
+    binding.decode_dense_ragged(dec.shape, dec.params, dw.q, dw.K, dw.V, seq, w.n, None, 0, dense_c, dec.ws)
     torch.cuda.synchronize()
     assert dec.device_status() == 0
+    orc_d = parity.oracle_rows(w, dw.q_host, dw.K_host, dw.V_host, meta, lens, tau_bh, dense=True)
+    parity.compare_rows(w, lens, None, dense_p, orc_d, check_lists=False)
     assert torch.equal(dense_c, dense_p)
 
 

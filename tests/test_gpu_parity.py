@@ -166,9 +166,16 @@ def test_edge_single_token_and_exact_blocks():
         _full_check(w, dense=True)
 
 
-def test_edge_n_local_and_offset():
-    w = _reduced(5).replace(n_local=3)
-    _full_check(w, 0.25)
+@pytest.mark.parametrize("cfg,n_local", [(5, 2), (5, 3), (3, 2), (6, 2)])
+def test_edge_n_local(cfg, n_local):
+    """More than one trailing block admitted unscreened (the pages' lwb = 2 of
+    Table 12's header, read as two local window blocks; 3 as a further case)."""
+    w = _reduced(cfg).replace(n_local=n_local)
+    r = _full_check(w, 0.25)
+    assert np.all(r["gpu"]["active_cnt"] >= n_local)
+
+
+def test_edge_offset():
     w = _reduced(3)
     _full_check(w, 0.38, offset_a=0.4)
     _full_check(w, 0.38, offset_a=-0.8)
@@ -302,56 +309,86 @@ def _sample_heads(w, k, seed=0):
     return sorted(pairs[i] for i in idx)
 
 
-def _full_size(w, density, n_out_heads, list_pairs=None):
-    """Full-size workload: every list/score/count checked on the given (b, kvh)
-    pairs (default all), outputs on sampled heads."""
-    dw = DeviceWorkload(w, keep_host=True)
+def _full_size(w, densities, list_pairs=None, streamed=False):
+    """Full-size workload in the benchmark's launch configuration: for each
+    density, every list, score, count and union on the given (b, kvh) pairs
+    (default all), thresholds bit-exact, and the outputs of every head of those
+    pairs, against the oracle. streamed: the cache is generated straight into
+    device memory and only the sampled batch rows are regenerated on the host
+    for the oracle (caches far larger than host memory needs)."""
+    if isinstance(densities, float):
+        densities = (densities,)
     pairs = list_pairs or [(b, h) for b in range(w.B) for h in range(w.Hkv)]
-    meta = parity.oracle_meta(w, dw.K_host, pairs)
+    if streamed:
+        dw = DeviceWorkload(w)
+        K_host, V_host = parity.host_rows(w, dw.q_host, [b for b, _ in pairs], dw.needles)
+    else:
+        dw = DeviceWorkload(w, keep_host=True)
+        K_host, V_host = dw.K_host, dw.V_host
+    meta = parity.oracle_meta(w, K_host, pairs)
     list_heads = [(b, kvh * w.G + g) for (b, kvh) in pairs for g in range(w.G)]
-    tau, stride, bias = parity.oracle_thresholds(w, dw.q_host, meta, density, W=dw.W, heads=list_heads)
-    gpu = parity.run_gpu(dw, tau, stride, bias=bias)
-    assert gpu["status"] == 0
-    if bias is not None:
-        assert np.array_equal(gpu["tau"].view(np.int32), np.asarray(tau, np.float32).view(np.int32))
-    out_heads = set(_sample_heads(w.replace(B=w.B), n_out_heads))
-    out_heads = sorted(h for h in out_heads if (h[0], h[1] // w.G) in set(pairs)) or list_heads[:2]
-    orc = parity.oracle_step(w, dw.q_host, dw.K_host, dw.V_host, meta, tau, stride, list_heads)
-    # lists for every head, outputs for all of them too (the oracle is threaded)
-    parity.compare(w, gpu, orc, list_heads)
-    dens = sum(int(gpu["active_cnt"][b, h]) for (b, h) in list_heads) / (len(list_heads) * w.nb)
-    return dens
+    got = []
+    for density in densities:
+        tau, stride, bias = parity.oracle_thresholds(w, dw.q_host, meta, density, W=dw.W, heads=list_heads)
+        gpu = parity.run_gpu(dw, tau, stride, bias=bias)
+        assert gpu["status"] == 0
+        if bias is not None:
+            assert np.array_equal(gpu["tau"].view(np.int32), np.asarray(tau, np.float32).view(np.int32))
+        orc = parity.oracle_step(w, dw.q_host, K_host, V_host, meta, tau, stride, list_heads)
+        parity.compare(w, gpu, orc, list_heads)
+        got.append(sum(int(gpu["active_cnt"][b, h]) for (b, h) in list_heads) / (len(list_heads) * w.nb))
+    return got[0] if len(got) == 1 else got
 
 
 def test_full_size_gqa_128k_bench_config():
+    """The benchmark's workload at its three densities (20 / 38 / 60% per head)."""
     w = synth.WORKLOADS[3]
     pairs = [(0, 0), (3, 5), (7, 7)]
-    dens = _full_size(w, 0.38, 0, list_pairs=pairs)
-    assert 0.3 < dens < 0.5
+    d20, d38, d60 = _full_size(w, (0.20, 0.38, 0.60), list_pairs=pairs)
+    assert 0.12 < d20 < 0.3 and 0.3 < d38 < 0.5 and 0.5 < d60 < 0.7
 
 
 def test_full_size_mha_32k_needles():
-    _full_size(synth.WORKLOADS[2], 0.38, 0)
+    _full_size(synth.WORKLOADS[2], 0.38)
 
 
 def test_full_size_512k_sampled():
     w = synth.WORKLOADS[4]
-    _full_size(w, 0.38, 0, list_pairs=[(0, 2), (0, 11)])
+    _full_size(w, 0.38, list_pairs=[(0, 2), (0, 11)])
 
 
 def test_full_size_64k_b16_batch16_sampled():
+    """The calibrated-constant sweep at batch 16: 10%, 25% and 100% (every block)."""
     w = synth.WORKLOADS[5].replace(B=16)
-    _full_size(w, 0.25, 0, list_pairs=[(0, 0), (9, 3), (15, 15)])
+    d10, d25, d100 = _full_size(w, (0.10, 0.25, 1.0), list_pairs=[(0, 0), (9, 3), (15, 15)])
+    assert d10 < d25 < d100 == 1.0
+
+
+def test_full_size_64k_b16_batch64_rows_past_2_31():
+    """The sweep's largest batch (64 rows, 32 GiB of K and V): the last rows'
+    element offsets exceed 2^31. Lists and outputs of rows 0, 31 and 63 against
+    the oracle at 38% and 60%."""
+    w = synth.WORKLOADS[5].replace(B=64)
+    assert ((63 * w.Hkv + 15) * w.capacity * w.d) > 2 ** 31
+    _full_size(w, (0.38, 0.60), list_pairs=[(0, 0), (31, 8), (63, 15)], streamed=True)
 
 
 def test_full_size_fp8_gqa_128k():
     """Workload 7 (the 128K GQA workload with fp8 K/V) at full size."""
     w = synth.WORKLOADS[7]
-    dens = _full_size(w, 0.38, 0, list_pairs=[(0, 0), (5, 3), (7, 7)])
+    dens = _full_size(w, 0.38, list_pairs=[(0, 0), (5, 3), (7, 7)])
     assert 0.3 < dens < 0.5
 
 
 def test_full_size_table10_shape_sampled():
     """The pages' Table 10 head shape (32/4 heads, d 64, b 64) at 512K tokens, batch 4."""
     w = synth.WORKLOADS[6].replace(B=4)
-    _full_size(w, 0.05, 0, list_pairs=[(0, 0), (3, 3)])
+    _full_size(w, 0.05, list_pairs=[(0, 0), (3, 3)])
+
+
+def test_full_size_table10_shape_batch64_rows_past_2_31():
+    """Table 10's own batch (64 rows of 512K tokens, 32 GiB of K and V): rows 0,
+    40 and 63 against the oracle, thresholds of every row bit-exact."""
+    w = synth.WORKLOADS[6]
+    assert w.B == 64 and ((63 * w.Hkv + 3) * w.capacity * w.d) > 2 ** 31
+    _full_size(w, (0.12, 0.25), list_pairs=[(0, 1), (40, 2), (63, 3)], streamed=True)

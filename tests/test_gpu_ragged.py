@@ -34,46 +34,11 @@ def _outs(w):
 
 
 def _oracle_rows(w, dw, meta, lens, tau_bh, dense=False):
-    qf = oracle.to_f32(dw.q_host)
-
-    def one(b, hq):
-        n_b = lens[b]
-        nb_b = (n_b + w.bs - 1) // w.bs
-        kvh = hq // w.G
-        if dense:
-            lst, sc = np.arange(nb_b, dtype=np.int32), None
-            t = float("-inf")
-        else:
-            mu, var, mx = meta[(b, kvh)]
-            t = tau_bh(b, hq)
-            lst, sc = oracle.screen_head(qf[b, hq], mu, var, mx, nb_b, w.n_local, w.z, t)
-        o = oracle.attend_head(dw.K_host[b, kvh], dw.V_host[b, kvh], w.bs, n_b, qf[b, hq], lst, t, w.beta)
-        return (b, hq), (lst, sc, o)
-    return dict(parity.pmap(one, [(b, h) for b in range(w.B) for h in range(w.Hq)]))
+    return parity.oracle_rows(w, dw.q_host, dw.K_host, dw.V_host, meta, lens, tau_bh, dense)
 
 
 def _compare(w, lens, outs, out, orc, check_lists=True):
-    tol = parity.TOL[w.dtype]
-    got = {k: v.cpu().numpy() for k, v in outs.items()} if check_lists else {}
-    o_gpu = out.cpu().numpy()
-    for (b, hq), (lst, sc, o) in orc.items():
-        err = float(np.max(np.abs(o_gpu[b, hq].astype(np.float64) - o)))
-        assert err <= tol, f"output of row {b} (n={lens[b]}) head {hq}: {err:.3g}"
-        if not check_lists:
-            continue
-        cnt = int(got["active_cnt"][b, hq])
-        assert cnt == len(lst) and np.array_equal(got["active_idx"][b, hq, :cnt], lst), (b, hq, lens[b])
-        ns_b = max(0, (lens[b] + w.bs - 1) // w.bs - w.n_local)
-        assert np.array_equal(got["scores"][b, hq, :ns_b].view(np.int32), sc.view(np.int32)), (b, hq)
-        assert np.all(np.isnan(got["scores"][b, hq, ns_b:w.n_screened])), "scores past the row were written"
-    for b in range(w.B):
-        nb_b = (lens[b] + w.bs - 1) // w.bs
-        for kvh in range(w.Hkv if check_lists else 0):
-            idx, mask = oracle.union_lists([orc[(b, kvh * w.G + g)][0] for g in range(w.G)], nb_b)
-            ucnt = int(got["union_cnt"][b, kvh])
-            packed = (idx.astype(np.int64) << 8) | mask.astype(np.int64)
-            assert ucnt == len(idx)
-            assert np.array_equal(got["union_list"][b, kvh, :ucnt].astype(np.int64) & 0xffffffff, packed)
+    parity.compare_rows(w, lens, outs, out, orc, check_lists)
 
 
 @pytest.mark.parametrize("dtype,Hq,Hkv,d,bs,mode", [
