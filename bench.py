@@ -49,6 +49,10 @@ def parse_args():
     p.add_argument("--impl", default="eta", choices=["eta", "reference"])
     p.add_argument("--config", type=int, default=3)
     p.add_argument("--batch", type=int, default=None, help="override the batch (config 5 sweep)")
+    p.add_argument("--seq-len", type=int, default=None, help="override the cached tokens per row")
+    p.add_argument("--cap-blocks", type=int, default=None,
+                   help="override the capacity per row, in blocks (not a multiple of 4: metadata rows that "
+                        "are not 16-byte aligned, screened with plain loads)")
     p.add_argument("--density", type=float, default=None,
                    help="target admitted fraction (default: the middle density of the workload)")
     p.add_argument("--n-splits", type=int, default=0)
@@ -72,6 +76,19 @@ def parse_args():
 
 
 # ----------------------------------------------------------------- plumbing
+def workload_of(args):
+    """The benchmark workload with the command line's overrides applied."""
+    from learned_block_sparse_b200 import synth
+    w = synth.WORKLOADS[args.config]
+    if args.batch:
+        w = w.replace(B=args.batch)
+    if args.seq_len:
+        w = w.replace(n=args.seq_len)
+    if args.cap_blocks:
+        w = w.replace(cap=args.cap_blocks * w.bs)
+    return w
+
+
 def relaunch_command(argv, n: int, port: int):
     """The torch.distributed.run command that starts n ranks of this script
     with the same arguments (one process per GPU, rendezvous on 127.0.0.1)."""
@@ -260,11 +277,15 @@ def byte_model(w, union_cnt: np.ndarray, head_cnt: np.ndarray, S: int, r: int = 
     kv = 2 * row * (blocks * w.bs - bh * (w.bs - last_rows))
     lists_read = 4 * blocks
     q = w.B * w.Hq * w.d * eb
-    T = blocks
+    # the decode splits ring positions over its thread blocks: a block is one
+    # position, or bs / 32 of them on the tensor-core path (bf16, fp8) at
+    # d = 128 for blocks of 64 and 128 tokens
+    nsub = max(1, w.bs // 32) if (w.dtype != "f32" and w.d == 128) else 1
+    T = blocks * nsub
     # split merge: a segment inside one range writes its output rows directly;
     # one crossing ranges writes one (m, l, o) partial per range and head (read
     # back once by the merging thread block, from L2)
-    pre = np.concatenate([[0], np.cumsum(union_cnt.reshape(-1))])
+    pre = nsub * np.concatenate([[0], np.cumsum(union_cnt.reshape(-1))])
     partial_rows = 0
     for i in range(bh):
         if T >= S:
@@ -361,9 +382,7 @@ def run_reference(args):
     if rank != 0:
         return
     from learned_block_sparse_b200 import synth
-    w = synth.WORKLOADS[args.config]
-    if args.batch:
-        w = w.replace(B=args.batch)
+    w = workload_of(args)
     rng = np.random.default_rng(0)
     groups_all = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     n_groups = min(8, len(groups_all))
@@ -413,9 +432,7 @@ def run_eta(args):
     from learned_block_sparse_b200 import binding, synth
     from learned_block_sparse_b200.workload import DeviceWorkload
 
-    w = synth.WORKLOADS[args.config]
-    if args.batch:
-        w = w.replace(B=args.batch)
+    w = workload_of(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     dw = DeviceWorkload(w, device=dev, n_splits=args.n_splits, sub_blocks=args.sub_blocks)
     dec = dw.dec

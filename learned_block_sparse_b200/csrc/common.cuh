@@ -126,7 +126,8 @@ __device__ __forceinline__ bool wait_value_bounded(volatile int* p, int v, volat
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (*p == v) return true;
-    if ((it & 63u) == 0) {
+    __nanosleep(32);  // back off: a polling warp takes no issue slots from the working ones
+    if ((it & 15u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;

@@ -298,7 +298,7 @@ cudaError_t launch_decode_t(const DecodeCall& c, cudaStream_t st) {
   cudaError_t e = allow_max_smem(smem_done, reinterpret_cast<const void*>(decode_kernel<KV, D, G, DENSE>));
   if (e != cudaSuccess) return e;
 
-  const DecodeArgs a = make_decode_args(c, nst);
+  const DecodeArgs a = make_decode_args(c, nst, s.block_size);  // one position per block
   return launch_pdl(decode_kernel<KV, D, G, DENSE>, static_cast<unsigned>(c.S), kDecThreads, smem, st, a);
 }
 

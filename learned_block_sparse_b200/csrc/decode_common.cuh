@@ -30,6 +30,9 @@ struct DecodeArgs {
   int B, Hq, Hkv, bs, nb, nb_cap, nstages, q_dtype;
   int gate;  // ETA_GATE_SIGMOID or ETA_GATE_HARD
   float beta, qscale;
+  // Ring positions: each admitted block is 2^sub_log2 positions of rpos rows
+  // (rpos = bs >> sub_log2); flat positions, ranges and segment bounds count them.
+  int sub_log2, rpos;
   int64_t withhold;  // test hook: position of thread block 0's range whose copy is never armed (-1: none)
 };
 
@@ -170,17 +173,19 @@ __device__ __forceinline__ void finish_segment(const DecodeArgs& a, int seg, int
   }
 }
 
-// Producer warp: walk positions [lo, hi) in order. Lanes 0..PL-1 each take
-// every PL-th position (position lo + i goes to lane i % PL; PL = kMaxPL, or
-// less when the ring has fewer stages, so PL consecutive positions never share
-// a stage and are armed in parallel): wait until the position's stage is free,
-// publish (block, head mask, rows, segment) in s_info and call
-// issue(stage, row0, rows) (row0: the block's first row in the [rows][d] view
-// of the K and V stores), which must arm s_full[stage] (arrive +
-// expected bytes) and start the copies. The warp reads the union list 32
-// entries at a time, one batch ahead. A stage's r-th reuse waits for the
-// consumer release that completed the empty barrier's phase r-1; the round a
-// stage serves is then published in s_round (when given) before it is armed.
+// Producer warp: walk positions [lo, hi) in order. A position is rows
+// [sub * rpos, (sub + 1) * rpos) of an admitted block, whose 2^sub_log2
+// positions are consecutive. Lanes 0..PL-1 each take every PL-th position
+// (position lo + i goes to lane i % PL; PL = kMaxPL, or less when the ring has
+// fewer stages, so PL consecutive positions never share a stage and are armed
+// in parallel): wait until the position's stage is free, publish
+// (block * 2^sub_log2 + sub, head mask, rows, segment) in s_info and call
+// issue(stage, row0, rows) (row0: the position's first row in the [rows][d]
+// view of the K and V stores), which must arm s_full[stage] (arrive + expected
+// bytes) and start the copies. The warp reads the union list 32 entries at a
+// time, one batch ahead. A stage's r-th reuse waits for the consumer release
+// that completed the empty barrier's phase r-1; the round a stage serves is
+// then published in s_round (when given) before it is armed.
 //
 // Abort protocol. Consumers release a stage only after its full barrier
 // completed, so a stage is never re-armed while its copies are in flight.
@@ -200,47 +205,53 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
   while (PL > NST) PL >>= 1;
   const int lane = threadIdx.x & 31;
   // entry of position p, in two halves so the list load of the next batch is
-  // in flight while this batch is issued: fetch() gives the segment and
-  // (block << 8 | head mask); finish() the block's rows (tokens of the row
-  // inside it; -1 when the block is past the row or its page outside the pool)
-  // and the store row of its token 0
-  auto fetch = [&](int64_t p, int& seg, uint32_t& e) {
+  // in flight while this batch is issued: fetch() gives the segment, the
+  // position's sub-block and (block << 8 | head mask); finish() its rows
+  // (tokens of the row inside it: 0 for a sub-block past the row's last token,
+  // -1 when the whole block is past the row or its page outside the pool) and
+  // the store row of its first token
+  auto fetch = [&](int64_t p, int& seg, int& sub, uint32_t& e) {
     seg = 0;
+    sub = 0;
     e = 0;
     if (p < hi) {
       seg = seg_of(p);
       const int64_t j = p - pre(seg);
-      e = DENSE ? ((static_cast<uint32_t>(j) << 8) | ((1u << G) - 1u))
-                : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + j);
+      const int64_t jb = j >> a.sub_log2;
+      sub = static_cast<int>(j - (jb << a.sub_log2));
+      e = DENSE ? ((static_cast<uint32_t>(jb) << 8) | ((1u << G) - 1u))
+                : __ldg(a.union_list + static_cast<int64_t>(seg) * a.nb_cap + jb);
     }
   };
-  auto finish = [&](int64_t p, int seg, uint32_t e, int& rows, int& row0) {
+  auto finish = [&](int64_t p, int seg, int sub, uint32_t e, int& rows, int& row0) {
     rows = 0;
     row0 = 0;
     if (p < hi) {
       const int blk = static_cast<int>(e >> 8);
-      const int64_t r = seg_tokens(a, seg) - static_cast<int64_t>(blk) * a.bs;
-      rows = r <= 0 ? -1 : (r < a.bs ? static_cast<int>(r) : a.bs);
+      const int64_t r = seg_tokens(a, seg) - static_cast<int64_t>(blk) * a.bs - static_cast<int64_t>(sub) * a.rpos;
+      rows = r > 0 ? (r < a.rpos ? static_cast<int>(r) : a.rpos) : (sub == 0 ? -1 : 0);
       if (rows > 0) {
         row0 = kv_block_row(a.kv, seg, blk);
         if (row0 < 0) rows = -1;
+        else row0 += sub * a.rpos;
       }
     }
   };
-  int seg_cur, seg_nxt = 0, rows_cur, row_cur;
+  int seg_cur, seg_nxt = 0, sub_cur, sub_nxt = 0, rows_cur, row_cur;
   uint32_t e_cur, e_nxt = 0;
-  fetch(lo + lane, seg_cur, e_cur);
+  fetch(lo + lane, seg_cur, sub_cur, e_cur);
   int issued = 0;    // this lane: 1 + the last position (relative to lo) it armed
   int held = -1;     // the position left unarmed by the test hook
   int aborted = 0;
   volatile int* abort_flag = s_abort;
   for (int64_t base = lo; base < hi && !aborted; base += 32) {
-    finish(base + lane, seg_cur, e_cur, rows_cur, row_cur);
-    if (base + 32 < hi) fetch(base + 32 + lane, seg_nxt, e_nxt);
+    finish(base + lane, seg_cur, sub_cur, e_cur, rows_cur, row_cur);
+    if (base + 32 < hi) fetch(base + 32 + lane, seg_nxt, sub_nxt, e_nxt);
     const int cnt = static_cast<int>(hi - base < 32 ? hi - base : int64_t{32});
     for (int s = 0; s < cnt && !aborted; s += PL) {
       const int src = s + (lane < PL ? lane : 0);
       const int seg_i = __shfl_sync(kFull, seg_cur, src);
+      const int sub_i = __shfl_sync(kFull, sub_cur, src);
       const uint32_t e_i = __shfl_sync(kFull, e_cur, src);
       const int rows_i = __shfl_sync(kFull, rows_cur, src);
       const int row_i = __shfl_sync(kFull, row_cur, src);
@@ -258,7 +269,7 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
             rows = 0;
           }
           if (s_round != nullptr) s_round[st] = round;  // this stage now serves round `round`
-          s_info[st] = make_int4(blk, static_cast<int>(e_i & 0xffu), rows, seg_i);
+          s_info[st] = make_int4((blk << a.sub_log2) + sub_i, static_cast<int>(e_i & 0xffu), rows, seg_i);
           if (blockIdx.x == 0 && it == a.withhold) held = it;   // test hook: never armed
           else if (rows == 0) mbar_arrive(&s_full[st]);
           else issue(st, row_i, rows);
@@ -268,6 +279,7 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
       aborted = __any_sync(kFull, aborted) ? 1 : 0;
     }
     seg_cur = seg_nxt;
+    sub_cur = sub_nxt;
     e_cur = e_nxt;
   }
   // Positions >= last - NST are the last armed use of their stage (last = 1 +
@@ -285,8 +297,9 @@ __device__ __forceinline__ void producer_loop(const DecodeArgs& a, int64_t lo, i
   }
 }
 
-// Host side: the arguments common to both decode kernels.
-inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
+// Host side: the arguments common to both decode kernels; positions of rpos
+// rows (the block size divided by a power of two).
+inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages, int rpos) {
   const eta_shape_t& s = c.shape;
   DecodeArgs a;
   a.k = c.k;
@@ -321,6 +334,9 @@ inline DecodeArgs make_decode_args(const DecodeCall& c, int nstages) {
   a.beta = c.beta;
   a.gate = c.gate;
   a.withhold = c.withhold;
+  a.rpos = rpos;
+  a.sub_log2 = 0;
+  while ((rpos << a.sub_log2) < s.block_size) ++a.sub_log2;
   a.qscale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(s.head_dim)));
   return a;
 }

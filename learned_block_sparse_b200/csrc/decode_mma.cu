@@ -206,8 +206,11 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int BH = a.B * a.Hkv;
   const int NST = a.nstages;
-  const int bs = a.bs;
-  const uint32_t tile_bytes = static_cast<uint32_t>(bs) * D * EB;
+  // a ring position is rp rows of an admitted block: the whole block, or at
+  // d = 128 a chunk of CH rows (a block of 64 or 128 tokens is 2 or 4
+  // positions), so a warp has the next chunk in flight while it attends one
+  const int rp = a.rpos, sl = a.sub_log2;
+  const uint32_t tile_bytes = static_cast<uint32_t>(rp) * D * EB;
   unsigned char* s_tiles = smem;
   uint64_t* s_full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(NST) * 2 * tile_bytes);
   uint64_t* s_empty = s_full + NST;
@@ -237,11 +240,12 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
   }
   __syncthreads();
 
+  // segment i's first position, and the segment of position p
   auto pre = [&](int i) -> int64_t {
-    return flat ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i]);
+    return (flat ? static_cast<int64_t>(i) * a.nb : static_cast<int64_t>(s_pre[i])) << sl;
   };
   auto seg_of = [&](int64_t p) -> int {
-    return flat ? static_cast<int>(p / a.nb) : find_seg(s_pre, BH, p);
+    return flat ? static_cast<int>((p >> sl) / a.nb) : find_seg(s_pre, BH, p >> sl);
   };
   const int64_t T = pre(BH);
   const int S = gridDim.x;
@@ -260,15 +264,15 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
       const int y = row0;
       unsigned char* kt = s_tiles + static_cast<size_t>(st) * 2 * tile_bytes;
       unsigned char* vt = kt + tile_bytes;
-      uint64_t* bar = rows == bs ? &s_full[st] : &s_aux[lane];
+      uint64_t* bar = rows == rp ? &s_full[st] : &s_aux[lane];
       mbar_arrive_expect_tx(bar, 2 * tile_bytes);
       constexpr int kBoxElems = 128 / EB;  // a box row is 128 bytes
 #pragma unroll
       for (int h = 0; h < D / kBoxElems; ++h) {
-        tma_load_2d(kt + h * bs * 128, &tmk, h * kBoxElems, y, bar, pol);
-        tma_load_2d(vt + h * bs * 128, &tmv, h * kBoxElems, y, bar, pol);
+        tma_load_2d(kt + h * rp * 128, &tmk, h * kBoxElems, y, bar, pol);
+        tma_load_2d(vt + h * rp * 128, &tmv, h * kBoxElems, y, bar, pol);
       }
-      if (rows == bs) return;
+      if (rows == rp) return;
       // Partial block: the store's rows past the row's last token may hold
       // anything, NaN included. Their keys are masked by the consumer, but
       // P = 0 times NaN would still reach O, so their values are zeroed here
@@ -279,9 +283,9 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
         }
       }
       aux_phase ^= 1u;
-      for (int r = rows; r < bs; ++r)
+      for (int r = rows; r < rp; ++r)
 #pragma unroll
-        for (int c = 0; c < D * EB / 16; ++c) *reinterpret_cast<uint4*>(vt + swz(bs, r, c)) = make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < D * EB / 16; ++c) *reinterpret_cast<uint4*>(vt + swz(rp, r, c)) = make_uint4(0u, 0u, 0u, 0u);
       // generic-proxy writes: order them before the next TMA write into the stage
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&s_full[st]);
@@ -390,11 +394,11 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     const uint32_t vt = kt + tile_bytes;
     const int rows = inf.z;
     const bool row_on = live_row && ((static_cast<uint32_t>(inf.y) >> row) & 1u);
-    const int64_t tok0 = static_cast<int64_t>(inf.x) * bs;
-    // full block that does not hold the current token: no per-key checks
-    const bool fast = rows == bs && tok0 + bs <= t_cur;
+    const int64_t tok0 = static_cast<int64_t>(inf.x) * rp;
+    // full position that does not hold the current token: no per-key checks
+    const bool fast = rows == rp && tok0 + rp <= t_cur;
     constexpr int NT = CH / 8;  // n-tiles of 8 keys per chunk
-    for (int c0 = 0; c0 < bs; c0 += CH) {
+    for (int c0 = 0; c0 < rp; c0 += CH) {
       // S = Q K^T: even and odd k-steps accumulate separately (shorter mma chains)
       float se[NT][2], so[NT][2];  // bf16: partial sums of the even and odd k-steps
       float sv[FP8 ? NT : 1][2];   // fp8: the scaled logits
@@ -410,7 +414,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
           uint32_t bb[NT][4];
 #pragma unroll
           for (int j = 0; j < NT; ++j)
-            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * u + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+            ldsm_x4(kt + swz(rp, c0 + 8 * j + (lane & 7), 4 * u + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
                     bb[j][3]);
 #pragma unroll
           for (int j = 0; j < NT; ++j) mma_16832_e4m3(sa[j], q8[2 * u], bb[j][0], bb[j][1]);
@@ -430,7 +434,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
           uint32_t bb[NT][4];
 #pragma unroll
           for (int j = 0; j < NT; ++j)
-            ldsm_x4(kt + swz(bs, c0 + 8 * j + (lane & 7), 4 * k2 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
+            ldsm_x4(kt + swz(rp, c0 + 8 * j + (lane & 7), 4 * k2 + (lane >> 3)), bb[j][0], bb[j][1], bb[j][2],
                     bb[j][3]);
 #pragma unroll
           for (int j = 0; j < NT; ++j)
@@ -516,7 +520,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
 #pragma unroll
           for (int g = 0; g < D / 16; g += 2) {
             uint32_t r0, r1, r2, r3;
-            ldsm_x4_t(vt + swz(bs, vrow, g + (lane >> 4)), r0, r1, r2, r3);
+            ldsm_x4_t(vt + swz(rp, vrow, g + (lane >> 4)), r0, r1, r2, r3);
             // each register: keys 2q, 2q+1 x dims 2c, 2c+1; regroup into the
             // even-dim and the odd-dim key pairs (bytes 0,2 and 1,3)
             uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
@@ -544,7 +548,7 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
 #pragma unroll
           for (int jd = 0; jd < NDT; jd += 2) {
             uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vt + swz(bs, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
+            ldsm_x4_t(vt + swz(rp, vrow, jd + (lane >> 4)), b0, b1, b2, b3);
             // A rows 0-7: high part, rows 8-15: low part of the same P row
             mma_16816(o[jd], h0, l0, h1, l1, b0, b1);
             mma_16816(o[jd + 1], h0, l0, h1, l1, b2, b3);
@@ -594,7 +598,10 @@ __global__ void __launch_bounds__(MmaWarps<D, CH, FP8>::kThreads, 1)
     // still be in flight), and the producer stops once it sees the abort
     ok = __all_sync(kFull, ok);
     if (ok) {
-      process(st, s_info[st]);
+      // a position with no rows (a chunk past its row's last token) loaded
+      // nothing: its stage holds stale data, so it is not attended
+      const int4 inf = s_info[st];
+      if (inf.z > 0) process(st, inf);
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_empty[st]);
     }
@@ -614,15 +621,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [rows][d] view of a K or V store (bf16, or fp8 bytes), boxes of [bs] rows of
-// 128 bytes with the 128-byte swizzle.
-bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int bs, bool fp8) {
+// [rows][d] view of a K or V store (bf16, or fp8 bytes), boxes of [box_rows]
+// rows of 128 bytes with the 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* tm, const void* base, int64_t rows, int d, int box_rows, bool fp8) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   const int eb = fp8 ? 1 : 2;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(d) * eb};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(bs)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estride[2] = {1u, 1u};
   return enc(tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
              gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -633,7 +640,12 @@ template <int D, int G, bool DENSE, int CH, bool FP8>
 cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;
   const int BH = s.batch * s.n_kv_heads;
-  const size_t tile = static_cast<size_t>(s.block_size) * D * (FP8 ? 1 : 2);
+  // rows per ring position: 32-row chunks of the blocks at d = 128 (a warp
+  // then has its next chunk in flight while it attends one: 36.9 -> 34.8 us on
+  // the 32K batch-1 decode), whole blocks at d = 64, whose 8 KB chunks cost
+  // more per position than they gain (1,738 -> 1,881 us on the Table 10 shape)
+  const int rp = D == 128 ? CH : s.block_size;
+  const size_t tile = static_cast<size_t>(rp) * D * (FP8 ? 1 : 2);  // one position of K (or V)
   constexpr int kMW = MmaWarps<D, CH, FP8>::kMW;
   constexpr unsigned kThreads = MmaWarps<D, CH, FP8>::kThreads;
   const size_t fixed = static_cast<size_t>(kMW) * G * (D + 2) * sizeof(float) + 16 + 8 * sizeof(uint64_t) +
@@ -653,10 +665,10 @@ cudaError_t launch_mma_t(const DecodeCall& c, cudaStream_t st) {
   CUtensorMap tmk, tmv;
   const int64_t rows = c.block_table != nullptr ? static_cast<int64_t>(c.num_pages) * s.n_kv_heads * s.block_size
                                                 : static_cast<int64_t>(BH) * s.capacity;
-  if (!encode_kv_map(&tmk, c.k, rows, D, s.block_size, FP8) || !encode_kv_map(&tmv, c.v, rows, D, s.block_size, FP8))
+  if (!encode_kv_map(&tmk, c.k, rows, D, rp, FP8) || !encode_kv_map(&tmv, c.v, rows, D, rp, FP8))
     return cudaErrorInvalidValue;
 
-  const DecodeArgs a = make_decode_args(c, nst);
+  const DecodeArgs a = make_decode_args(c, nst, rp);
   if (c.gate == ETA_GATE_HARD) {
     static std::atomic<uint64_t> smem_done{0};
     const void* fn = reinterpret_cast<const void*>(decode_mma_kernel<D, G, DENSE, CH, true, FP8>);

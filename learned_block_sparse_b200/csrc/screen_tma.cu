@@ -5,12 +5,16 @@
 // head), lane = block, all G heads of the group per metadata read). Here a
 // producer warp streams each 32-block tile's metadata, one 2-D box of
 // [d coordinates][32 blocks] of mu and one of var (32 KB at d = 128), into a
-// ring of shared-memory stages; consumer warp w scores tiles w, w + CW, ... from
-// shared memory (lane = column, so the reads are conflict-free) with the
-// multiply-adds in increasing coordinate order. The ring keeps several tiles in
-// flight per SM even when a (batch, kv head) has few tiles, which plain loads
-// from a handful of warps cannot. The stage count is a multiple of the consumer
-// count, so a stage always returns to the warp that released it.
+// ring of shared-memory stages; consumer warps take the tiles in increasing
+// order from a shared counter and score them from shared memory (lane =
+// column, so the reads are conflict-free) with the multiply-adds in increasing
+// coordinate order. The warps that form the Eq. 1 thresholds join the
+// consumers once the thresholds are in (at once without a predictor). The ring
+// keeps several tiles in flight per SM even when a (batch, kv head) has few
+// tiles, which plain loads from a handful of warps cannot. Since any warp may
+// take any tile, the producer publishes the round each stage serves (after the
+// stage's previous release) and a consumer waits for its tile's round before
+// the barrier parity wait, which is then exact.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -24,20 +28,25 @@ namespace eta {
 
 namespace {
 
+// 96 KB of stages: two thread blocks per SM. (Measured and not kept: each
+// tile's coordinates as two ring positions of half the size, so a warp frees
+// half a stage before it has scored the whole tile and twice as many warps
+// score at once: 63 against 64 us at d = 128, G = 4; 301 against 279 us at
+// d = 64, G = 8.)
 template <int D> struct TmaScreenCfg;
-// 96 KB of stages: two thread blocks per SM.
 template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 3; };
 template <> struct TmaScreenCfg<64> { static constexpr int kCW = 3, kNST = 6; };
 // Warps that form the Eq. 1 thresholds (when the call passes a predictor)
-// while the ring streams the first tiles: the consumers score tiles and
-// release their stages without waiting for them, and wait only before the
-// first admission decision.
+// while the ring streams the first tiles, then score tiles too: the first
+// consumers score tiles and release their stages without waiting for the
+// thresholds, and wait only before their first admission decision.
 constexpr int kTauWarps = 4;
 
 // Bytes between the stages and ScreenSmem: full and empty barriers, the
-// threshold barrier (+ 8 bytes padding), the abort flag (+ 12 bytes padding).
+// threshold barrier (+ 8 bytes padding), the abort flag, the tile counter
+// (+ 8 bytes padding), the round of every stage (padded to 16 bytes).
 template <int NST>
-constexpr size_t kTmaBarBytes = (2 * NST + 2) * sizeof(uint64_t) + 4 * sizeof(int);
+constexpr size_t kTmaBarBytes = (2 * NST + 2) * sizeof(uint64_t) + (4 + (NST + 3) / 4 * 4) * sizeof(int);
 
 __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* tm, int x, int y, uint64_t* bar) {
   asm volatile(
@@ -47,8 +56,8 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
       : "memory");
 }
 
-// Packed fp32 pairs: fma.rn.f32x2 performs two independent IEEE fused
-// multiply-adds, each rounding as __fmaf_rn does.
+// Packed fp32 pairs: fma.rn.f32x2 / mul.rn.f32x2 perform two independent IEEE
+// fused multiply-adds / multiplies, each rounding as __fmaf_rn / __fmul_rn do.
 __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
   uint64_t r;
   asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
@@ -56,6 +65,11 @@ __device__ __forceinline__ uint64_t pack2(float lo, float hi) {
 }
 __device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b) {
   asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 __device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
@@ -69,7 +83,6 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   constexpr int NST = TmaScreenCfg<D>::kNST;
   constexpr int NT = (CW + 1 + kTauWarps) * 32;  // consumers, producer, threshold warps
   constexpr uint32_t kBox = D * 32 * sizeof(float);  // one array's tile
-  static_assert(NST % CW == 0, "stages must return to the same consumer warp");
   cg::cluster_group cluster = cg::this_cluster();
   const int cs = static_cast<int>(cluster.num_blocks());
   const int cr = static_cast<int>(cluster.block_rank());
@@ -85,6 +98,8 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   uint64_t* s_empty = s_full + NST;
   uint64_t* s_tau = s_empty + NST;  // completes when the thresholds are in sm.taut
   int* s_abort = reinterpret_cast<int*>(s_tau + 2);
+  int* s_next = s_abort + 1;     // next tile to hand out
+  int* s_round = s_abort + 4;    // [NST] round each stage serves
   // the query rows are read as float4: ScreenSmem must start 16-byte aligned
   static_assert((static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>) % 16 == 0, "ScreenSmem alignment");
   const ScreenSmem<D, G> sm(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>, tpc);
@@ -93,9 +108,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
 
   if (tid == 0) {
     *s_abort = 0;
+    *s_next = 0;
     for (int s = 0; s < NST; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
+      s_round[s] = 0;
     }
     mbar_init(s_tau, 1);
     fence_mbar_init();
@@ -125,38 +142,25 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   screen_prologue<D, G, 32, false>(a, sm, b, kvh, NT);  // ends with __syncthreads
   const bool tau_later = a.W != nullptr;
 
-  if (warp > CW) {
-    // ----------------------------------------------------- threshold warps
-    if (tau_later) {
-      constexpr int kTauThreads = kTauWarps * 32;
-      screen_predict_tau<D, G, 32>(a, sm, b, kvh, tid - (CW + 1) * 32, kTauThreads,
-                                   [] { named_barrier_sync(2, kTauThreads); });
-      named_barrier_sync(2, kTauThreads);  // every taut written before the release
-      if (tid == (CW + 1) * 32) mbar_arrive(s_tau);
-    }
-  } else if (warp == CW) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      volatile int* abort_flag = s_abort;
-      for (int it = first; it < my_tiles; ++it) {
-        const int st = it % NST, round = it / NST;
-        // a consumer that gave up does not release its stage: stop arming
-        if (!mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status) || *abort_flag) break;
-        issue_tile(it);
-        issued = it + 1;
-      }
-    }
-  } else {
-    // ----------------------------------------------------------- consumers
-    bool tau_ok = !tau_later;
-    bool tau_waited = !tau_later;
-    for (int it = warp; it < my_tiles; it += CW) {
-      const int st = it % NST;
+  // Consumers: take tiles in increasing order until none is left. tau_ready:
+  // the thresholds are in sm.taut already (no wait before the decisions).
+  auto consume = [&](bool tau_ready) {
+    bool tau_ok = tau_ready;
+    bool tau_waited = tau_ready;
+    volatile int* rounds = s_round;
+    for (;;) {
+      int it = 0;
+      if (lane == 0) it = atomicAdd(s_next, 1);
+      it = __shfl_sync(kFull, it, 0);
+      if (it >= my_tiles) break;
       const int unit = (t0 + it) * 32 + lane;
       const bool valid = unit < units;
       const float M = __ldg(mx + (valid ? unit : units - 1));  // units >= 1 here (this CTA has a tile)
-      const bool ok =
-          __all_sync(kFull, mbar_wait_bounded(&s_full[st], static_cast<uint32_t>((it / NST) & 1), s_abort, status));
+      // the stage serves this tile once the producer has published its round
+      // (after the previous round's release): the parity wait is then exact
+      const int st = it % NST, round = it / NST;
+      bool ok = round == 0 || wait_value_bounded(rounds + st, round, s_abort, status);
+      ok = __all_sync(kFull, ok && mbar_wait_bounded(&s_full[st], static_cast<uint32_t>(round & 1), s_abort, status));
       float dg[G], vg[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) dg[g] = vg[g] = 0.0f;
@@ -178,13 +182,14 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
           }
         } else {
           // heads 2p and 2p+1 share a packed multiply-add per coordinate: the
-          // [D][G] query rows give both of a coordinate's factors in one load
+          // [D][G] query rows give both of a coordinate's factors in one load,
+          // and fl(q q) of both in one packed multiply (the prologue's squares,
+          // bit for bit), which saves the shared loads of the squares
           const uint64_t* q2 = reinterpret_cast<const uint64_t*>(sm.q);
-          const uint64_t* qq2 = reinterpret_cast<const uint64_t*>(sm.qq);
           uint64_t d2[G / 2], v2[G / 2];
 #pragma unroll
           for (int p = 0; p < G / 2; ++p) d2[p] = v2[p] = 0ull;  // +0.0f in both halves
-#pragma unroll 2
+#pragma unroll 4
           for (int i0 = 0; i0 < D; i0 += 4) {
             float m[4], v[4];
 #pragma unroll
@@ -197,8 +202,9 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
               const uint64_t mm = pack2(m[c], m[c]), vv = pack2(v[c], v[c]);
 #pragma unroll
               for (int p = 0; p < G / 2; ++p) {
-                fma2(d2[p], q2[(i0 + c) * (G / 2) + p], mm);
-                fma2(v2[p], qq2[(i0 + c) * (G / 2) + p], vv);
+                const uint64_t qp = q2[(i0 + c) * (G / 2) + p];
+                fma2(d2[p], qp, mm);
+                fma2(v2[p], mul2(qp, qp), vv);
               }
             }
           }
@@ -217,6 +223,35 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
       }
       screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, unit, valid && tau_ok, dg, vg, M));
     }
+  };
+
+  if (warp > CW) {
+    // ----------------------------------------------------- threshold warps
+    if (tau_later) {
+      constexpr int kTauThreads = kTauWarps * 32;
+      screen_predict_tau<D, G, 32>(a, sm, b, kvh, tid - (CW + 1) * 32, kTauThreads,
+                                   [] { named_barrier_sync(2, kTauThreads); });
+      named_barrier_sync(2, kTauThreads);  // every taut written before the release
+      if (tid == (CW + 1) * 32) mbar_arrive(s_tau);
+    }
+    consume(true);  // then score tiles like the other consumers
+  } else if (warp == CW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      volatile int* abort_flag = s_abort;
+      volatile int* rounds = s_round;
+      for (int it = first; it < my_tiles; ++it) {
+        const int st = it % NST, round = it / NST;
+        // a consumer that gave up does not release its stage: stop arming
+        if (!mbar_wait_bounded(&s_empty[st], (round - 1) & 1, s_abort, status) || *abort_flag) break;
+        rounds[st] = round;  // this stage now serves round `round`
+        issue_tile(it);
+        issued = it + 1;
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- consumers
+    consume(!tau_later);
   }
   __syncthreads();
   if (warp == CW && lane == 0 && *reinterpret_cast<volatile int*>(s_abort)) {
@@ -245,13 +280,13 @@ PFN_cuTensorMapEncodeTiled_v12000 meta_map_encoder() {
 }
 
 // [rows][ncol] fp32 view of mu or var (ncol metadata columns: blocks, or
-// sub-blocks with the envelope), boxes of [d rows][32 columns].
-bool encode_meta_map(CUtensorMap* tm, const float* base, int64_t rows, int64_t nb_cap, int d) {
+// sub-blocks with the envelope), boxes of [box_rows coordinates][32 columns].
+bool encode_meta_map(CUtensorMap* tm, const float* base, int64_t rows, int64_t nb_cap, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = meta_map_encoder();
   if (enc == nullptr) return false;
   const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(nb_cap), static_cast<cuuint64_t>(rows)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(nb_cap) * sizeof(float)};
-  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(d)};
+  const cuuint32_t box[2] = {32u, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estride[2] = {1u, 1u};
   return enc(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), gdim, gstride, box, estride,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -268,7 +303,9 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   const int ns = max(0, nb - c.n_local);
   const int nt = (ns * c.sub_blocks + 31) / 32;
   // Clusters as large as keeps the launch within one wave of two thread blocks
-  // per SM (at least 1, at most kMaxCluster, at most one tile per CTA).
+  // per SM (at least 1, at most kMaxCluster, at most one tile per CTA). (Larger
+  // clusters that would balance SMs holding one and two thread blocks measured
+  // slower: 191 against 172 us on 256 pairs of 128 tiles.)
   int cs = static_cast<int>((2 * static_cast<int64_t>(device_sm_count())) / BH);
   cs = max(1, min(cs, min(kMaxCluster, nt)));
   while ((nt + cs - 1) / cs > kMaxScreenTiles && cs < kMaxCluster) ++cs;

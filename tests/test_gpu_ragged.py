@@ -138,10 +138,12 @@ def test_graph_replay_reads_the_new_lengths():
 
 
 @pytest.mark.parametrize("dtype,d,bs", [("bf16", 128, 32), ("bf16", 128, 16), ("bf16", 64, 64), ("f32", 64, 16),
-                                        ("fp8", 128, 32)])
+                                        ("fp8", 128, 32), ("bf16", 128, 128), ("fp8", 128, 64), ("bf16", 64, 128)])
 def test_cache_rows_past_each_length_are_never_used(dtype, d, bs):
     """Tokens at or past a row's length (the rest of its last block and beyond)
-    may hold anything: filling them with NaN changes no output bit."""
+    may hold anything: filling them with NaN changes no output bit. With blocks
+    of 64 and 128 tokens the tensor-core decode loads a block as chunks of 32
+    rows, and whole chunks past a row's end are never loaded nor attended."""
     w = synth.Workload("tail", dtype, 5, 8, 2, d, bs * 40 + 9, bs, z=1.0, tau_mode="const",
                        densities=(0.3,), seed=900 + bs + d, offset_std=synth.SQRT_HALF)
     dw = DeviceWorkload(w)
