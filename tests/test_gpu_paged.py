@@ -61,6 +61,7 @@ def _outs(w):
     ("bf16", 4, 4, 128, 16, "const"),
     ("f32", 4, 2, 64, 16, "predictor"),
     ("fp8", 8, 2, 128, 64, "const"),
+    ("bf16", 8, 2, 128, 128, "predictor"),  # four 32-row ring positions per page
 ])
 def test_paged_pool_against_oracle_and_contiguous_cache(dtype, Hq, Hkv, d, bs, mode):
     w = synth.Workload("paged", dtype, 6, Hq, Hkv, d, bs * 50 + 3, bs, z=1.0, tau_mode=mode,

@@ -47,6 +47,9 @@ def _compare(w, lens, outs, out, orc, check_lists=True):
     ("bf16", 4, 4, 128, 16, "const"),       # 16-token blocks, 8-warp decode
     ("f32", 4, 2, 64, 16, "predictor"),     # CUDA-core decode
     ("fp8", 8, 2, 128, 32, "const"),        # fp8 K/V
+    ("bf16", 16, 4, 128, 64, "predictor"),  # d = 128: a block is two 32-row ring positions
+    ("bf16", 8, 2, 128, 128, "const"),      # four positions per block, whole ones past a row's end
+    ("fp8", 8, 2, 128, 64, "predictor"),
 ])
 def test_ragged_rows_match_per_row_oracle(dtype, Hq, Hkv, d, bs, mode):
     w = synth.Workload("ragged", dtype, 7, Hq, Hkv, d, bs * 70 + 9, bs, z=1.0, tau_mode=mode,
