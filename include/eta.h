@@ -385,6 +385,24 @@ ETA_API eta_status_t eta_block_stats(const eta_shape_t* shape, const eta_params_
                                      float* block_max, int32_t* above, float* block_lse, eta_stream_t stream);
 
 /*
+ * eta_screen_diagnostics — Table 16's screen quality per query head, from the
+ * outputs of eta_block_stats (block_max, above, block_lse) and of eta_screen
+ * (active_idx, active_cnt) for the same shape, params, n_tokens and tau. Over
+ * a head's screened blocks j < ceil(n_tokens / b) - n_local, a block is "truly
+ * active" when block_max[j] >= fl(tau - a):
+ *   per_head[b][h][0] false negatives: truly active blocks not admitted / truly active
+ *   per_head[b][h][1] false positives: admitted blocks not truly active / admitted
+ *   per_head[b][h][2] token recall:    sum of above over admitted blocks / over all
+ *   per_head[b][h][3] missed mass:     sum of exp(block_lse) over rejected blocks /
+ *                                      over every block (fp64)
+ * A zero denominator counts as one. per_head: [B][Hq][4] fp64, 8-byte aligned.
+ */
+ETA_API eta_status_t eta_screen_diagnostics(const eta_shape_t* shape, const eta_params_t* params, int64_t n_tokens,
+                                            const float* tau, int64_t tau_batch_stride, const float* block_max,
+                                            const int32_t* above, const float* block_lse, const int32_t* active_idx,
+                                            const int32_t* active_cnt, double* per_head, eta_stream_t stream);
+
+/*
  * eta_decode_sparse_static — eta_decode_sparse without a caller workspace and
  * without any device allocation. The paper has no counterpart: this entry
  * point exists for callers that cannot allocate device memory when they

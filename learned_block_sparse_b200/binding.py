@@ -105,6 +105,8 @@ def _load():
     L.eta_decode_dense_paged.argtypes = [P(Shape), P(Params), vp, vp, vp, Pages, vp, i64, vp, i64, vp, vp, sz, vp]
     L.eta_block_stats.restype = st
     L.eta_block_stats.argtypes = [P(Shape), P(Params), vp, vp, i64, vp, i64, vp, vp, vp, vp]
+    L.eta_screen_diagnostics.restype = st
+    L.eta_screen_diagnostics.argtypes = [P(Shape), P(Params), i64, vp, i64, vp, vp, vp, vp, vp, vp, vp]
     L.eta_test_withhold_copy.restype = st
     L.eta_test_withhold_copy.argtypes = [i64]
     L.eta_decode_screened.restype = st
@@ -126,7 +128,7 @@ EXPORTED = ("eta_abi_version", "eta_status_string", "eta_build_block_meta", "eta
             "eta_screen_predict", "eta_decode_sparse_predict", "eta_screen_ragged", "eta_decode_sparse_ragged",
             "eta_decode_screened_ragged", "eta_decode_dense_ragged", "eta_build_block_meta_paged",
             "eta_decode_sparse_paged", "eta_decode_screened_paged", "eta_decode_dense_paged", "eta_block_stats",
-            "eta_test_withhold_copy")
+            "eta_screen_diagnostics", "eta_test_withhold_copy")
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
@@ -360,6 +362,16 @@ def decode_sparse_static(shape: Shape, params: Params, q, k, v, meta, n_tokens: 
                                         Meta(*(m.data_ptr() for m in meta)), n_tokens, _ptr(tau), tau_batch_stride,
                                         _ptr(out), ctypes.byref(so) if so is not None else None,
                                         _ptr(device_status), _stream(stream)), "eta_decode_sparse_static")
+
+
+def screen_diagnostics(shape: Shape, params: Params, n_tokens: int, tau: torch.Tensor, tau_batch_stride: int,
+                       block_max: torch.Tensor, above: torch.Tensor, block_lse: torch.Tensor,
+                       active_idx: torch.Tensor, active_cnt: torch.Tensor, per_head: torch.Tensor,
+                       stream=None) -> None:
+    _check(lib.eta_screen_diagnostics(ctypes.byref(shape), ctypes.byref(params), n_tokens, _ptr(tau),
+                                      tau_batch_stride, _ptr(block_max), _ptr(above), _ptr(block_lse),
+                                      _ptr(active_idx), _ptr(active_cnt), _ptr(per_head), _stream(stream)),
+           "eta_screen_diagnostics")
 
 
 def withhold_next_copy(position: int) -> None:

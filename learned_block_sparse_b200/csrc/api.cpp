@@ -593,6 +593,35 @@ ETA_API eta_status_t eta_decode_dense_paged(const eta_shape_t* shape, const eta_
                    stream, true, seq_lens, &pages);
 }
 
+ETA_API eta_status_t eta_screen_diagnostics(const eta_shape_t* shape, const eta_params_t* params, int64_t n_tokens,
+                                            const float* tau, int64_t tau_batch_stride, const float* block_max,
+                                            const int32_t* above, const float* block_lse, const int32_t* active_idx,
+                                            const int32_t* active_cnt, double* per_head, eta_stream_t stream) {
+  ETA_TRY(check_shape(shape));
+  ETA_TRY(check_params(params));
+  ETA_TRY(check_tokens(shape, n_tokens));
+  if (tau == nullptr || tau_batch_stride < 0 || block_max == nullptr || above == nullptr || block_lse == nullptr ||
+      active_idx == nullptr || active_cnt == nullptr || per_head == nullptr)
+    return ETA_ERR_INVALID_ARG;
+  if (!aligned(tau, 4) || !aligned(block_max, 4) || !aligned(above, 4) || !aligned(block_lse, 4) ||
+      !aligned(active_idx, 4) || !aligned(active_cnt, 4) || !aligned(per_head, 8))
+    return ETA_ERR_INVALID_ARG;
+  DiagCall c;
+  c.shape = *shape;
+  c.n = n_tokens;
+  c.n_local = params->n_local;
+  c.offset_a = params->offset_a;
+  c.tau = tau;
+  c.tau_stride = tau_batch_stride;
+  c.bmax = block_max;
+  c.above = above;
+  c.blse = block_lse;
+  c.active_idx = active_idx;
+  c.active_cnt = active_cnt;
+  c.out = per_head;
+  return from_cuda(launch_screen_diagnostics(c, stream));
+}
+
 ETA_API eta_status_t eta_test_withhold_copy(int64_t position) {
   g_withhold.store(position < 0 ? -1 : position);
   return ETA_OK;

@@ -132,6 +132,22 @@ struct StatsCall {
 };
 cudaError_t launch_block_stats(const StatsCall& c, cudaStream_t st);
 
+struct DiagCall {
+  eta_shape_t shape;
+  int64_t n;
+  int n_local;
+  float offset_a;
+  const float* tau;
+  int64_t tau_stride;
+  const float* bmax;        // [B][Hq][nb_cap]
+  const int32_t* above;     // [B][Hq][nb_cap]
+  const float* blse;        // [B][Hq][nb_cap]
+  const int32_t* active_idx;  // [B][Hq][nb_cap]
+  const int32_t* active_cnt;  // [B][Hq]
+  double* out;              // [B][Hq][4]
+};
+cudaError_t launch_screen_diagnostics(const DiagCall& c, cudaStream_t st);
+
 // Largest B*Hkv the decode kernel's on-chip prefix table holds.
 constexpr int kMaxBH = 8192;
 // The workspace starts with a fixed header, the part that must be zero before

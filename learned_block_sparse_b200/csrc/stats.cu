@@ -131,7 +131,114 @@ cudaError_t launch_stats_d(const StatArgs& a, int BH, int G, cudaStream_t st) {
   }
 }
 
+// Table 16's screen diagnostics of one query head (one warp per head), from
+// its block statistics and its ascending admitted list, over the ns screened
+// blocks (the forced trailing blocks excluded); a block is truly active when
+// its max scaled logit reaches fl(tau - a):
+//   false_negative = truly active blocks not admitted / truly active blocks
+//   false_positive = admitted blocks not truly active / admitted blocks
+//   token_recall   = tokens at or above fl(tau - a) in admitted blocks / all such tokens
+//   missed_mass    = gated softmax mass of the rejected blocks over that of all nb blocks
+// Counts are exact; the masses are fp64 sums of exp(lse_j - max lse) in a fixed
+// order (lane-strided partials, then a butterfly), so the result does not
+// depend on timing. A zero denominator counts as one (the ratio is then 0).
+struct DiagArgs {
+  const float* tau;
+  int64_t tau_stride;
+  const float* bmax;
+  const int32_t* above;
+  const float* blse;
+  const int32_t* active_idx;
+  const int32_t* active_cnt;
+  double* out;  // [B][Hq][4]
+  float offset_a;
+  int heads, Hq, nb, ns, nb_cap;
+};
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kStatThreads) diag_kernel(const DiagArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int hd = static_cast<int>(blockIdx.x) * (kStatThreads / 32) + (threadIdx.x >> 5);  // b * Hq + h
+  if (hd >= a.heads) return;
+  const int b = hd / a.Hq, h = hd - b * a.Hq;
+  const float ts = __fsub_rn(a.tau[b * a.tau_stride + h], a.offset_a);
+  const int64_t row = static_cast<int64_t>(hd) * a.nb_cap;
+  const float* bm = a.bmax + row;
+  const int32_t* ab = a.above + row;
+  const float* ls = a.blse + row;
+  double mx = -INFINITY;
+  for (int j = lane; j < a.nb; j += 32) mx = fmax(mx, static_cast<double>(ls[j]));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) mx = fmax(mx, __shfl_xor_sync(kFull, mx, o));
+  const double base = mx == -INFINITY ? 0.0 : mx;
+  // every block: the normaliser; screened blocks: active count, tokens, mass
+  double all = 0.0, scr = 0.0, act = 0.0, tok = 0.0;
+  for (int j = lane; j < a.nb; j += 32) {
+    const double e = exp(static_cast<double>(ls[j]) - base);
+    all += e;
+    if (j < a.ns) {
+      scr += e;
+      act += bm[j] >= ts ? 1.0 : 0.0;
+      tok += static_cast<double>(ab[j]);
+    }
+  }
+  // the admitted screened blocks
+  const int cnt = a.active_cnt[hd];
+  const int32_t* lst = a.active_idx + row;
+  double adm = 0.0, both = 0.0, tok_adm = 0.0, mass_adm = 0.0;
+  for (int k = lane; k < cnt; k += 32) {
+    const int j = lst[k];
+    if (j < 0 || j >= a.ns) continue;
+    adm += 1.0;
+    both += bm[j] >= ts ? 1.0 : 0.0;
+    tok_adm += static_cast<double>(ab[j]);
+    mass_adm += exp(static_cast<double>(ls[j]) - base);
+  }
+  all = warp_sum(all);
+  scr = warp_sum(scr);
+  act = warp_sum(act);
+  tok = warp_sum(tok);
+  adm = warp_sum(adm);
+  both = warp_sum(both);
+  tok_adm = warp_sum(tok_adm);
+  mass_adm = warp_sum(mass_adm);
+  if (lane == 0) {
+    double* o = a.out + static_cast<int64_t>(hd) * 4;
+    o[0] = (act - both) / fmax(1.0, act);
+    o[1] = (adm - both) / fmax(1.0, adm);
+    o[2] = tok_adm / fmax(1.0, tok);
+    o[3] = (a.ns - adm) > 0.0 && all > 0.0 ? fmax(0.0, scr - mass_adm) / all : 0.0;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_screen_diagnostics(const DiagCall& c, cudaStream_t st) {
+  const eta_shape_t& s = c.shape;
+  DiagArgs a;
+  a.tau = c.tau;
+  a.tau_stride = c.tau_stride;
+  a.bmax = c.bmax;
+  a.above = c.above;
+  a.blse = c.blse;
+  a.active_idx = c.active_idx;
+  a.active_cnt = c.active_cnt;
+  a.out = c.out;
+  a.offset_a = c.offset_a;
+  a.heads = s.batch * s.n_q_heads;
+  a.Hq = s.n_q_heads;
+  a.nb = static_cast<int>((c.n + s.block_size - 1) / s.block_size);
+  a.ns = a.nb > c.n_local ? a.nb - c.n_local : 0;
+  a.nb_cap = static_cast<int>(s.capacity / s.block_size);
+  const unsigned grid = static_cast<unsigned>((a.heads + kStatThreads / 32 - 1) / (kStatThreads / 32));
+  diag_kernel<<<grid, kStatThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_stats(const StatsCall& c, cudaStream_t st) {
   const eta_shape_t& s = c.shape;

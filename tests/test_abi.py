@@ -124,6 +124,13 @@ def test_argument_validation_before_launch():
                                         None) == 2
     assert L.eta_build_block_meta_paged(ctypes.byref(s), a16, binding.Pages(1 << 20, 64), 0, 0, meta, None) == 0
     assert L.eta_predict_tau(ctypes.byref(s), None, a16, a16, a16, None) == 1
+    # screen diagnostics: every buffer required, the fp64 output 8-byte aligned
+    assert L.eta_screen_diagnostics(ctypes.byref(s), ctypes.byref(p), 100, a16, 0, a16, a16, a16, None, a16, a16,
+                                    None) == 1
+    assert L.eta_screen_diagnostics(ctypes.byref(s), ctypes.byref(p), 100, a16, 0, a16, a16, a16, a16, a16,
+                                    ctypes.c_void_p((1 << 20) + 4), None) == 1
+    assert L.eta_screen_diagnostics(ctypes.byref(s), ctypes.byref(p), 0, a16, 0, a16, a16, a16, a16, a16, a16,
+                                    None) == 1
     st = ctypes.c_int(0)
     assert L.eta_read_device_status(None, None, ctypes.byref(st)) == 1
     assert L.eta_workspace_init(bad, 1 << 20, None) == 3
