@@ -199,8 +199,9 @@ with open(sys.argv[3], "w", buffering=1) as f:
 class ClockSampler:
     """SM clock and clock-event reasons sampled DURING the timed region.
 
-    A separate process polls NVML about once a millisecond (an NVML query
-    takes ~1 us) and stamps each sample with the system-wide monotonic clock;
+    A separate process polls NVML every 0.2 ms (an NVML query takes ~1 us;
+    the shortest timed regions, a few steps of the tiny workload, last about
+    half a millisecond) and stamps each sample with the system-wide monotonic clock;
     start() returns once it is sampling, stop() keeps the samples taken between
     the two calls. A separate process, so the benchmark's own thread never
     delays the sampling. The device is found by its UUID (CUDA and NVML may
@@ -208,7 +209,7 @@ class ClockSampler:
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, device_index: int, period_s: float = 0.001):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
         self.dev = device_index
         self.period = period_s
         self.proc = None
@@ -262,7 +263,7 @@ class ClockSampler:
         sm = [x[0] for x in samples]
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in samples), "sm_mhz_min": min(sm),
                 "reasons": reasons, "samples": len(sm),
-                "source": "NVML polled ~1 kHz by a separate process, samples inside the timed region"}
+                "source": "NVML polled every 0.2 ms by a separate process, samples inside the timed region"}
 
 
 # ------------------------------------------------------------ byte models

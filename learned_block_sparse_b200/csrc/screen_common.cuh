@@ -82,10 +82,10 @@ struct ScreenSmem {
     tcnt = base + 16;
     mask = reinterpret_cast<uint8_t*>(tcnt + tpc * (G + 1));
   }
-  static constexpr size_t fixed_bytes() {
+  __host__ __device__ static constexpr size_t fixed_bytes() {
     return (2 * G * D + 48 + 32 * (G + 1)) * sizeof(float) + 32 * sizeof(int);
   }
-  static size_t bytes(int tpc) {
+  __host__ __device__ static size_t bytes(int tpc) {
     return fixed_bytes() + static_cast<size_t>(tpc) * (G + 1) * sizeof(int) + static_cast<size_t>(tpc) * 32;
   }
 };
@@ -153,17 +153,14 @@ __device__ __forceinline__ void screen_prologue(const ScreenArgs& a, const Scree
   __syncthreads();
 }
 
-// Eq. 5 for one metadata unit and every head of the group, given the
+// Eq. 5 scores of one metadata unit for every head of the group, given the
 // fma-accumulated D = sum q_i mu_i and V = sum q_i^2 var_i; with sub-blocks
 // (r > 1) the block's score is the largest over its r units, which sit in r
 // consecutive lanes (r divides 32, and the r units of a block are all valid or
-// all invalid); the first of them decides the block. Writes the scores (if
-// asked) and returns the head mask of the admitted heads. All 32 lanes call it.
+// all invalid). Independent of the thresholds. All 32 lanes call it.
 template <int D, int G>
-__device__ __forceinline__ uint32_t screen_decide(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
-                                                  int unit, bool valid, const float (&dg)[G], const float (&vg)[G],
-                                                  float M) {
-  float sc[G];
+__device__ __forceinline__ void screen_scores(const ScreenArgs& a, const ScreenSmem<D, G>& sm, const float (&dg)[G],
+                                              const float (&vg)[G], float M, float (&sc)[G]) {
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const float A = __fadd_rn(dg[g], __fmul_rn(a.z, __fsqrt_rn(vg[g])));
@@ -174,8 +171,16 @@ __device__ __forceinline__ uint32_t screen_decide(const ScreenArgs& a, const Scr
     for (int o = 1; o < a.r; o <<= 1)
 #pragma unroll
       for (int g = 0; g < G; ++g) sc[g] = fmaxf(sc[g], __shfl_xor_sync(kFull, sc[g], o));
-    valid = valid && (threadIdx.x & (a.r - 1)) == 0;
   }
+}
+
+// The admission rule on the scores of one unit (with sub-blocks the first unit
+// of a block decides it): writes the scores (if asked) and returns the head
+// mask of the admitted heads. All 32 lanes call it.
+template <int D, int G>
+__device__ __forceinline__ uint32_t screen_admit(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
+                                                 int unit, bool valid, const float (&sc)[G]) {
+  if (a.r > 1) valid = valid && (threadIdx.x & (a.r - 1)) == 0;
   const int blk = unit / a.r;
   uint32_t mask = 0;
 #pragma unroll
@@ -184,6 +189,16 @@ __device__ __forceinline__ uint32_t screen_decide(const ScreenArgs& a, const Scr
     if (a.scores != nullptr && valid) a.scores[(static_cast<int64_t>(b) * a.Hq + kvh * G + g) * a.nb_cap + blk] = sc[g];
   }
   return mask;
+}
+
+// Eq. 5 and the admission rule for one unit: screen_scores, then screen_admit.
+template <int D, int G>
+__device__ __forceinline__ uint32_t screen_decide(const ScreenArgs& a, const ScreenSmem<D, G>& sm, int b, int kvh,
+                                                  int unit, bool valid, const float (&dg)[G], const float (&vg)[G],
+                                                  float M) {
+  float sc[G];
+  screen_scores<D, G>(a, sm, dg, vg, M, sc);
+  return screen_admit<D, G>(a, sm, b, kvh, unit, valid, sc);
 }
 
 // Record one tile's masks and admission counts (one warp, lane = block).

@@ -9,7 +9,9 @@
 // order from a shared counter and score them from shared memory (lane =
 // column, so the reads are conflict-free) with the multiply-adds in increasing
 // coordinate order. The warps that form the Eq. 1 thresholds join the
-// consumers once the thresholds are in (at once without a predictor). The ring
+// consumers once the thresholds are in (at once without a predictor); tiles
+// scored before then keep their scores in shared memory and are decided after
+// the last tile, so the ring does not wait for the thresholds. The ring
 // keeps several tiles in flight per SM even when a (batch, kv head) has few
 // tiles, which plain loads from a handful of warps cannot. Since any warp may
 // take any tile, the producer publishes the round each stage serves (after the
@@ -28,23 +30,36 @@ namespace eta {
 
 namespace {
 
-// 96 KB of stages: two thread blocks per SM. (Measured and not kept: each
-// tile's coordinates as two ring positions of half the size, so a warp frees
-// half a stage before it has scored the whole tile and twice as many warps
-// score at once: 63 against 64 us at d = 128, G = 4; 301 against 279 us at
-// d = 64, G = 8.)
+// 96 KB of stages at d = 128, 80 KB at d = 64: with the per-tile bookkeeping
+// of up to 256 tiles, two thread blocks fit per SM (six stages at d = 64 left
+// one thread block per SM: 279 against 236 us on the Table 10 shape). (Measured
+// and not kept: each tile's coordinates as two ring positions of half the
+// size, so a warp frees half a stage before it has scored the whole tile and
+// twice as many warps score at once: 63 against 64 us at d = 128, G = 4; 301
+// against 279 us at d = 64, G = 8. And one flat split of all pairs' tiles
+// over the resident thread blocks, with the list offsets passed between them
+// in global memory: 72 against 66 us at d = 128, G = 4, 238 against 236 us on
+// the Table 10 shape; the SMs' unequal shares of the bandwidth, not the
+// tiles per SM, set the finish.)
 template <int D> struct TmaScreenCfg;
 template <> struct TmaScreenCfg<128> { static constexpr int kCW = 3, kNST = 3; };
-template <> struct TmaScreenCfg<64> { static constexpr int kCW = 3, kNST = 6; };
+template <> struct TmaScreenCfg<64> { static constexpr int kCW = 3, kNST = 5; };
 // Warps that form the Eq. 1 thresholds (when the call passes a predictor)
 // while the ring streams the first tiles, then score tiles too: the first
 // consumers score tiles and release their stages without waiting for the
 // thresholds, and wait only before their first admission decision.
 constexpr int kTauWarps = 4;
+// Tiles whose Eq. 5 scores may wait in shared memory for the thresholds: the
+// consumers score and release a stage before the Eq. 1 thresholds are in and
+// decide those tiles after the last one, instead of stalling the ring. Fewer
+// at d = 128, G = 8, where shared memory is tightest.
+template <int D, int G>
+constexpr int kTmaDefer = (D == 128 && G == 8) ? 4 : 8;
 
 // Bytes between the stages and ScreenSmem: full and empty barriers, the
-// threshold barrier (+ 8 bytes padding), the abort flag, the tile counter
-// (+ 8 bytes padding), the round of every stage (padded to 16 bytes).
+// threshold barrier (+ 8 bytes padding), the abort flag, the tile counter, the
+// deferred-tile count (+ 4 bytes padding), the round of every stage (padded to
+// 16 bytes).
 template <int NST>
 constexpr size_t kTmaBarBytes = (2 * NST + 2) * sizeof(uint64_t) + (4 + (NST + 3) / 4 * 4) * sizeof(int);
 
@@ -54,6 +69,17 @@ __device__ __forceinline__ void tma_load_2d_plain(void* dst, const CUtensorMap* 
           smem_u32(dst)),
       "l"(tm), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Non-blocking: has the phase of `bar` with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 // Packed fp32 pairs: fma.rn.f32x2 / mul.rn.f32x2 perform two independent IEEE
@@ -99,16 +125,22 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
   uint64_t* s_tau = s_empty + NST;  // completes when the thresholds are in sm.taut
   int* s_abort = reinterpret_cast<int*>(s_tau + 2);
   int* s_next = s_abort + 1;     // next tile to hand out
+  int* s_ndefer = s_abort + 2;   // tiles deferred
   int* s_round = s_abort + 4;    // [NST] round each stage serves
   // the query rows are read as float4: ScreenSmem must start 16-byte aligned
   static_assert((static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>) % 16 == 0, "ScreenSmem alignment");
   const ScreenSmem<D, G> sm(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST>, tpc);
+  constexpr int ND = kTmaDefer<D, G>;
+  float* s_defer = reinterpret_cast<float*>(smem + static_cast<size_t>(NST) * 2 * kBox + kTmaBarBytes<NST> +
+                                            ScreenSmem<D, G>::bytes(tpc));  // [ND][G][32] scores
+  int* s_defer_it = reinterpret_cast<int*>(s_defer + ND * G * 32);          // [ND] their tiles
 
   const float* mx = a.maxn + static_cast<int64_t>(bh) * a.nb_cap_meta;
 
   if (tid == 0) {
     *s_abort = 0;
     *s_next = 0;
+    *s_ndefer = 0;
     for (int s = 0; s < NST; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
@@ -144,9 +176,11 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
 
   // Consumers: take tiles in increasing order until none is left. tau_ready:
   // the thresholds are in sm.taut already (no wait before the decisions).
+  // Before they are in, a tile's scores go to a free deferral slot; with none
+  // free, the warp waits for them.
   auto consume = [&](bool tau_ready) {
-    bool tau_ok = tau_ready;
-    bool tau_waited = tau_ready;
+    bool tau_ok = true;
+    bool tau_have = tau_ready;
     volatile int* rounds = s_round;
     for (;;) {
       int it = 0;
@@ -217,11 +251,23 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
       }
       __syncwarp();
       if (ok && lane == 0) mbar_arrive(&s_empty[st]);  // a stage whose wait failed is not released
-      if (!tau_waited) {
+      float sc[G];
+      screen_scores<D, G>(a, sm, dg, vg, M, sc);
+      if (!tau_have && __all_sync(kFull, mbar_test_wait(s_tau, 0u))) tau_have = true;
+      if (!tau_have) {
+        int slot = 0;
+        if (lane == 0) slot = atomicAdd(s_ndefer, 1);
+        slot = __shfl_sync(kFull, slot, 0);
+        if (slot < ND) {
+#pragma unroll
+          for (int g = 0; g < G; ++g) s_defer[(slot * G + g) * 32 + lane] = sc[g];
+          if (lane == 0) s_defer_it[slot] = it;
+          continue;
+        }
         tau_ok = mbar_wait_bounded(s_tau, 0u, s_abort, status);
-        tau_waited = true;
+        tau_have = true;
       }
-      screen_record_tile<D, G>(sm, it, screen_decide<D, G>(a, sm, b, kvh, unit, valid && tau_ok, dg, vg, M));
+      screen_record_tile<D, G>(sm, it, screen_admit<D, G>(a, sm, b, kvh, unit, valid && tau_ok, sc));
     }
   };
 
@@ -263,6 +309,18 @@ __global__ void __launch_bounds__((TmaScreenCfg<D>::kCW + 1 + kTauWarps) * 32, 2
       }
     }
   }
+  // Deferred tiles: the thresholds are in (the threshold warps arrived before
+  // they joined the consumers, all of which are past the barrier above).
+  const int nd = min(*reinterpret_cast<volatile int*>(s_ndefer), ND);
+  for (int slot = warp; slot < nd; slot += NT / 32) {
+    const int it = s_defer_it[slot];
+    const int unit = (t0 + it) * 32 + lane;
+    float sc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) sc[g] = s_defer[(slot * G + g) * 32 + lane];
+    screen_record_tile<D, G>(sm, it, screen_admit<D, G>(a, sm, b, kvh, unit, unit < units, sc));
+  }
+  __syncthreads();
   screen_finish<D, G>(a, sm, b, kvh, bh, t0, my_tiles, rb, NT);
 }
 
@@ -312,7 +370,7 @@ cudaError_t launch_tma_t(const ScreenCall& c, cudaStream_t st) {
   const int tpc = max(1, (nt + cs - 1) / cs);
   if (tpc > kMaxScreenTiles) return cudaErrorInvalidValue;
   const size_t smem = 128 + static_cast<size_t>(NST) * 2 * D * 32 * sizeof(float) + kTmaBarBytes<NST> +
-                      ScreenSmem<D, G>::bytes(tpc);
+                      ScreenSmem<D, G>::bytes(tpc) + kTmaDefer<D, G> * (G * 32 * sizeof(float) + sizeof(int));
   if (smem > static_cast<size_t>(device_max_smem_optin())) return cudaErrorNotSupported;
   CUtensorMap tmu, tvar;
   const int64_t rows = static_cast<int64_t>(BH) * D;
